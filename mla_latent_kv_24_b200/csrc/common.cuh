@@ -1,0 +1,65 @@
+// Shared device helpers for libmla kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/mla.h"
+
+namespace mla {
+
+// ---------------------------------------------------------------------------------------
+// Device error word: kernels never trap; they record the first error code and skip the
+// offending access.  The host reads and clears it in mla_get_device_status().
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void report(int *err, int code) {
+    if (err) atomicCAS(err, 0, code);
+}
+
+// ---------------------------------------------------------------------------------------
+// Storage types.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// RoPE angle for pair i of a d-wide vector at position pos: pos * base^(-2i/d), with the
+// product and the trigonometry in double precision so that large positions (2^17) keep
+// full single-precision accuracy after rounding.
+__device__ __forceinline__ void rope_cos_sin(int pos, int i, int d, float base, float *c, float *s) {
+    double theta = pow((double)base, -2.0 * (double)i / (double)d);
+    double ang = (double)pos * theta;
+    double sd, cd;
+    sincos(ang, &sd, &cd);
+    *c = (float)cd;
+    *s = (float)sd;
+}
+
+__host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------------------------------
+// Split-KV plan.  Row r = (b, j) has len_r = seq_lens[b] - s_q + j + 1 visible tokens and
+// is cut into ceil(len_r / chunk) chunks of `chunk` tokens (the last one ragged).  Work item
+// k covers tokens [t0, t1) of one row; partial results are stored at index k.
+// ---------------------------------------------------------------------------------------
+struct WorkItem {
+    int row;     // b * s_q + j
+    int t0, t1;  // token range
+    int split;   // chunk index inside the row
+};
+
+struct Plan {
+    const WorkItem *items;  // [n_work]
+    const int *row_first;   // [rows + 1] first work item of each row (prefix sums)
+    int n_work;
+    int rows;
+    int chunk;
+};
+
+}  // namespace mla

@@ -1,0 +1,25 @@
+// Tensor-core decode kernels: the tcgen05 absorbed decode (decode_tc.cu) and the grouped
+// (GQA-path) decode (decode_grouped.cu).
+#pragma once
+
+#include "kernels.h"
+
+namespace mla {
+
+// Absorbed path, bf16, H=128, d_c=512, d_rope=64, page 64.
+bool tc_available();
+int tc_units(int sms);        // concurrent workers the split plan should cover
+int tc_token_granule();       // chunk lengths are multiples of this many tokens
+cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *latent, const int *page_table,
+                             const Plan &plan, int max_pages, int n_pages, int s_q, float *part_o,
+                             float *part_ml, int *err, int sms, cudaStream_t st);
+
+// Grouped path, bf16, d_nope = d_v = 128, d_rope = 64, heads_per_group = 8.
+bool grouped_tc_ok(const Dims &d);
+int grouped_units(const Dims &d, int sms);
+int grouped_token_granule();
+cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expanded, const void *latent,
+                                  const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
+                                  int n_pages, int s_q, float *part_o, float *part_ml, int *err, cudaStream_t st);
+
+}  // namespace mla

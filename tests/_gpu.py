@@ -1,0 +1,122 @@
+"""Helpers for the GPU parity tests: upload seeded inputs, call the C ABI through the binding,
+and compare with the oracle under the stated tolerances."""
+import numpy as np
+import torch
+
+import mla_latent_kv_24_b200 as mla
+import workloads as wl
+
+# bf16 inputs, fp32 accumulation: normwise max relative error and mean absolute error.
+BF16_REL, BF16_MAE = 1e-2, 1e-3
+FP32_REL = 1e-5
+
+
+def dims_of(w: wl.Workload):
+    return mla.make_dims(n_heads=w.H, heads_per_group=w.hpw, d_c=w.d_c, d_rope=w.d_r, d_nope=w.d_n, d_v=w.d_v,
+                         page_size=w.page, softmax_scale=w.softmax_scale, rope_base=w.rope_base, dtype=w.dtype)
+
+
+class Dev:
+    """Device copies of one workload's inputs."""
+
+    def __init__(self, inp: wl.DecodeInputs, device="cuda"):
+        self.inp = inp
+        w = inp.w
+        self.q = wl.to_torch(inp.q, device)
+        self.W_uk = wl.to_torch(inp.W_uk, device)
+        self.W_uv = wl.to_torch(inp.W_uv, device)
+        self.cache = wl.to_torch(inp.cache, device)
+        self.page_table = torch.from_numpy(inp.page_table).to(device)
+        self.seq_lens = torch.from_numpy(inp.seq_lens).to(device)
+        self.max_pages = inp.page_table.shape[1]
+        self.dims = dims_of(w)
+        self.tdtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def decode_absorbed(self, out=None, lens_host=None):
+        w = self.inp.w
+        lens_host = self.inp.seq_lens if lens_host is None else lens_host
+        nb = mla.mla_decode_workspace_size(self.dims, w.B, w.s_q, self.inp.seq_lens)
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=self.q.device)
+        out = torch.empty((w.B, w.s_q, w.H, w.d_v), dtype=self.tdtype, device=self.q.device) if out is None else out
+        mla.mla_decode_absorbed(self.dims, self.q, self.W_uk, self.W_uv, self.cache, self.page_table, self.seq_lens,
+                                lens_host, w.B, w.s_q, self.max_pages, self.inp.n_pages, out, ws)
+        return out
+
+    def expand(self):
+        w = self.inp.w
+        G = w.H // w.hpw
+        exp = torch.empty((self.inp.n_pages, G, w.page, w.d_n + w.d_v), dtype=self.tdtype, device=self.q.device)
+        mla.gqla_expand_cache(self.dims, self.W_uk, self.W_uv, self.cache, None, 0, self.inp.n_pages, exp)
+        return exp
+
+    def decode_grouped(self, expanded):
+        w = self.inp.w
+        nb = mla.gqla_decode_workspace_size(self.dims, w.B, w.s_q, self.inp.seq_lens)
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=self.q.device)
+        out = torch.empty((w.B, w.s_q, w.H, w.d_v), dtype=self.tdtype, device=self.q.device)
+        mla.gqla_decode_grouped(self.dims, self.q, expanded, self.cache, self.page_table, self.seq_lens,
+                                self.inp.seq_lens, w.B, w.s_q, self.max_pages, self.inp.n_pages, out, ws)
+        return out
+
+
+def errors(got: np.ndarray, ref: np.ndarray):
+    """(normwise max relative error, mean absolute error) over the finite entries of ref."""
+    m = np.isfinite(ref)
+    g, r = got[m], ref[m]
+    d = np.abs(g - r)
+    return float(d.max() / np.abs(r).max()), float(d.mean())
+
+
+def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
+    assert np.isfinite(got[np.isfinite(ref)]).all(), f"{what}: non-finite GPU output"
+    rel, mae = errors(got, ref)
+    if dtype == "bf16":
+        assert rel <= BF16_REL and mae <= BF16_MAE, f"{what}: rel {rel:.3e} mae {mae:.3e}"
+    else:
+        assert rel <= FP32_REL, f"{what}: rel {rel:.3e} mae {mae:.3e}"
+    return rel, mae
+
+
+def oracle_decode(inp: wl.DecodeInputs, sample=None):
+    import oracle
+    w = inp.w
+    return oracle.decode_expanded(inp.q.f64(), inp.W_uk.f64(), inp.W_uv.f64(), inp.cache.f64(), inp.page_table,
+                                  inp.seq_lens, w.hpw, w.softmax_scale, w.rope_base, sample=sample)
+
+
+def sample_outputs(inp: wl.DecodeInputs, n: int, seed: int = 99):
+    """n distinct (b, j, h) output rows, always including the longest request and the last head."""
+    w = inp.w
+    rng = np.random.default_rng(seed)
+    picks = {(int(np.argmax(inp.seq_lens)), w.s_q - 1, w.H - 1), (0, 0, 0)}
+    while len(picks) < n:
+        picks.add((int(rng.integers(w.B)), int(rng.integers(w.s_q)), int(rng.integers(w.H))))
+    return sorted(picks)
+
+
+def oracle_decode_sampled(inp: wl.DecodeInputs, sample):
+    """Oracle outputs for the sampled (b, j, h) rows only, converting just the cache rows of the
+    sampled requests to float64 (full-size caches do not fit in memory as float64)."""
+    import oracle
+    w = inp.w
+    q = inp.q.f64()
+    W_uk, W_uv = inp.W_uk.f64(), inp.W_uv.f64()
+    out = {}
+    for b in sorted({s[0] for s in sample}):
+        L = int(inp.seq_lens[b])
+        n = (L + w.page - 1) // w.page
+        bits = inp.cache.data[inp.page_table[b, :n]].reshape(n * w.page, w.d_row)[:L]
+        rows = wl.bf16_bits_to_f64(bits) if w.dtype == "bf16" else bits.astype(np.float64)
+        sel = [(j, h) for (bb, j, h) in sample if bb == b]
+        res = oracle.decode_request_expanded(q[b], rows, W_uk, W_uv, w.hpw, w.softmax_scale, w.rope_base,
+                                             heads=sorted({h for _, h in sel}), queries=sorted({j for j, _ in sel}))
+        for j, h in sel:
+            out[(b, j, h)] = res[j, h]
+    return out
+
+
+def compare_sampled(got: np.ndarray, ref: dict, dtype: str, what: str):
+    keys = sorted(ref)
+    g = np.stack([got[k] for k in keys])
+    r = np.stack([ref[k] for k in keys])
+    return assert_close(g, r, dtype, what)

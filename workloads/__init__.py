@@ -226,3 +226,17 @@ def new_token_positions(lens: np.ndarray, s_q: int):
 __all__ = ["Workload", "WORKLOADS", "DecodeInputs", "make_inputs", "Tensor", "PAGE",
            "f32_to_bf16_bits", "bf16_bits_to_f64", "bf16_bits_to_f32", "small_workload",
            "new_token_positions", "seq_lens", "page_table"]
+
+
+def to_torch(t: Tensor, device="cuda"):
+    """Copies a host tensor to torch (bf16 bit patterns become torch.bfloat16)."""
+    import torch
+    if t.dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(t.data).view(np.int16)).to(device).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(t.data)).to(device)
+
+
+def from_torch_f64(x) -> np.ndarray:
+    """Exact float64 copy of a torch tensor (bf16 or fp32) on any device."""
+    import torch
+    return x.detach().to("cpu", torch.float64).numpy()
