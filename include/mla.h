@@ -197,6 +197,35 @@ MLA_API mla_status gqla_decode_grouped(const mla_dims *dims, const void *q, cons
 MLA_API mla_status mla_get_device_status(mla_stream_t stream);
 
 /*
+ * mla_decode_absorbed_noalloc — mla_decode_absorbed for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this entry point; it changes where scratch lives,
+ * not what is computed.
+ *
+ * Some callers have no way to obtain a workspace: an engine whose memory manager has already
+ * reserved the whole device for its KV-cache pool and forbids ad-hoc cudaMalloc, or a
+ * latency-critical loop where cudaMalloc/cudaFree would stall on an implicit device
+ * synchronisation.  This variant takes the same inputs and output as mla_decode_absorbed but no
+ * workspace: its scratch is a static device array of MLA_NOALLOC_SCRATCH_BYTES compiled into
+ * the library, which every GPU that loads the library holds until the process exits.
+ *   - Returns MLA_ERR_WORKSPACE (nothing enqueued) when the batch needs more scratch than that;
+ *     mla_decode_workspace_size() tells how much a batch needs.
+ *   - The first call on a device looks up that device's address of the array (no allocation);
+ *     make the first call on each device before any stream capture.
+ *   - All calls share the one array, and every call rewrites what it reads from it, so nothing
+ *     needs clearing; but two calls that overlap on the GPU (different streams, or different
+ *     host threads, without ordering between them) race on it and corrupt each other.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (32u << 20)
+MLA_API mla_status mla_decode_absorbed_noalloc(const mla_dims *dims, const void *q, const void *W_uk,
+                                               const void *W_uv, const void *latent_cache,
+                                               const int32_t *page_table, const int32_t *seq_lens,
+                                               const int32_t *seq_lens_host, int32_t batch,
+                                               int32_t s_q, int32_t max_pages,
+                                               int32_t n_pages_total, void *out,
+                                               mla_stream_t stream);
+
+/*
  * mla_set_profile_events — measurement hook.  When both are non-NULL, every later
  * mla_decode_absorbed / gqla_decode_grouped call on the calling thread records `start_event`
  * on its stream immediately before launching its main attention kernel and `stop_event`

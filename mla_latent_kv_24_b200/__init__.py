@@ -19,7 +19,7 @@ __all__ = [
     "mla_cache_append", "mla_decode_workspace_size", "mla_decode_absorbed",
     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
     "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
-    "EXPORTED_SYMBOLS",
+    "mla_decode_absorbed_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so")
@@ -30,7 +30,9 @@ MLA_BF16, MLA_FP32 = 0, 1
 
 EXPORTED_SYMBOLS = ["mla_cache_append", "mla_decode_workspace_size", "mla_decode_absorbed",
                     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
-                    "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events"]
+                    "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
+                    "mla_decode_absorbed_noalloc"]
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class MlaError(RuntimeError):
@@ -78,6 +80,7 @@ def load() -> ctypes.CDLL:
         "mla_last_error_string": [],
         "mla_version": [],
         "mla_set_profile_events": [_P, _P],
+        "mla_decode_absorbed_noalloc": [D, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -179,3 +182,14 @@ def mla_set_profile_events(start=None, stop=None) -> None:
     s = None if start is None else ctypes.c_void_p(start.cuda_event)
     e = None if stop is None else ctypes.c_void_p(stop.cuda_event)
     _check(load().mla_set_profile_events(s, e))
+
+
+def mla_decode_absorbed_noalloc(dims, q, W_uk, W_uv, latent_cache, page_table, seq_lens, seq_lens_host, batch, s_q,
+                                max_pages, n_pages_total, out, stream=None) -> None:
+    """mla_decode_absorbed without a workspace argument, for callers that cannot allocate device
+    memory: the library's own static scratch (NOALLOC_SCRATCH_BYTES per device) is used.  Calls
+    that overlap on the GPU race on that scratch; batches that need more raise MlaError."""
+    arr, p = _host_i32(seq_lens_host)
+    _check(load().mla_decode_absorbed_noalloc(ctypes.byref(dims), _dev(q), _dev(W_uk), _dev(W_uv), _dev(latent_cache),
+                                              _dev(page_table), _dev(seq_lens), p, batch, s_q, max_pages,
+                                              n_pages_total, _dev(out), _stream(stream)))

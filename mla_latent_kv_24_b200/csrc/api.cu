@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <string>
 
 #include "kernels.h"
@@ -335,6 +336,52 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
         MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, L.DV, nullptr, out, st), "launch combine");
     }
     return MLA_OK;
+}
+
+// Scratch of mla_decode_absorbed_noalloc: a file-scope device array, so callers that cannot
+// allocate still get a workspace.  Host code must not use its name as an address (that names a
+// host-side stand-in); each device's real address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
+static void *g_noalloc_ptr[MAX_DEVICES];
+static std::mutex g_noalloc_mu;
+
+// Device address of the static scratch on the current device, looked up once per device.
+static mla_status noalloc_scratch(void **ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= MAX_DEVICES) return fail(MLA_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return MLA_OK;
+}
+
+mla_status mla_decode_absorbed_noalloc(const mla_dims *dims, const void *q, const void *W_uk, const void *W_uv,
+                                       const void *latent_cache, const int32_t *page_table,
+                                       const int32_t *seq_lens, const int32_t *seq_lens_host, int32_t batch,
+                                       int32_t s_q, int32_t max_pages, int32_t n_pages_total, void *out,
+                                       mla_stream_t stream) {
+    g_last_error.clear();
+    size_t need = 0;
+    Layout L;
+    MLA_TRY(decode_workspace(dims, ABSORBED, batch, s_q, seq_lens_host, &need, &L));
+    if (need > (size_t)MLA_NOALLOC_SCRATCH_BYTES)
+        return fail(MLA_ERR_WORKSPACE,
+                    "this batch needs %zu bytes of scratch; the static scratch of the no-allocation entry point "
+                    "holds %zu (use mla_decode_absorbed with a workspace)",
+                    need, (size_t)MLA_NOALLOC_SCRATCH_BYTES);
+    void *ws = nullptr;
+    MLA_TRY(noalloc_scratch(&ws));
+    return run_decode(ABSORBED, dims, q, W_uk, W_uv, latent_cache, nullptr, page_table, seq_lens, seq_lens_host,
+                      batch, s_q, max_pages, n_pages_total, out, ws, MLA_NOALLOC_SCRATCH_BYTES,
+                      (cudaStream_t)stream);
 }
 
 mla_status mla_decode_absorbed(const mla_dims *dims, const void *q, const void *W_uk, const void *W_uv,
