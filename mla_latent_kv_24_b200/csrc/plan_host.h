@@ -8,16 +8,36 @@
 
 namespace mla {
 
+inline long long plan_count(const int32_t *lens, int batch, int s_q, int chunk);
+
 // Chunk length (a multiple of `granule` tokens) that spreads all rows' tokens over about
-// `units` concurrently running workers.
+// `units` concurrently running workers: the smallest such length whose chunk count fits in
+// one wave of `units` when that is possible (more chunks than workers would leave a second,
+// mostly idle wave), otherwise the even split of all tokens.
 inline int plan_chunk(const int32_t *lens, int batch, int s_q, int units, int granule) {
-    long long total = 0;
+    long long total = 0, longest = 1;
     for (int b = 0; b < batch; ++b)
-        for (int j = 0; j < s_q; ++j) total += (long long)lens[b] - s_q + j + 1;
-    long long c = (total + units - 1) / std::max(1, units);
-    c = (c + granule - 1) / granule * granule;
-    c = std::max<long long>(c, granule);
-    return (int)std::min<long long>(c, 1 << 30);
+        for (int j = 0; j < s_q; ++j) {
+            const long long len = (long long)lens[b] - s_q + j + 1;
+            total += len;
+            longest = std::max(longest, len);
+        }
+    units = std::max(1, units);
+    auto round_up = [&](long long c) { return std::max<long long>(granule, (c + granule - 1) / granule * granule); };
+    long long lo = round_up((total + units - 1) / units);
+    long long hi = round_up(longest);
+    if (lo >= hi) return (int)std::min<long long>(lo, 1 << 30);
+    if (plan_count(lens, batch, s_q, (int)std::min<long long>(hi, 1 << 30)) > units)
+        return (int)std::min<long long>(lo, 1 << 30);
+    while (lo < hi) {  // smallest multiple of granule in [lo, hi] with count <= units
+        const long long mid = round_up((lo + hi) / 2 - granule + 1);
+        const long long m = mid < lo ? lo : mid;
+        if (plan_count(lens, batch, s_q, (int)m) <= units)
+            hi = m;
+        else
+            lo = m + granule;
+    }
+    return (int)std::min<long long>(lo, 1 << 30);
 }
 
 inline long long plan_count(const int32_t *lens, int batch, int s_q, int chunk) {

@@ -146,5 +146,8 @@ def test_request_alone_equals_request_in_batch():
         sub.inp = wl.DecodeInputs(**{**inp.__dict__, "seq_lens": inp.seq_lens[b:b + 1],
                                      "page_table": inp.page_table[b:b + 1], "w": wl.small_workload(w, B=1)})
         one = wl.from_torch_f64(sub.decode_absorbed())
-        d = np.abs(one[0] - full[b]).max() / np.abs(full[b]).max()
-        assert d <= 2e-3, d
+        # Different batches get different split plans, so fp32 sums run in another order and a
+        # bf16 output may move by an ulp; anything beyond two ulps of the largest value is a bug.
+        diff = np.abs(one[0] - full[b])
+        assert diff.max() / np.abs(full[b]).max() <= 2 ** -6, diff.max()
+        assert diff.mean() <= 1e-4, diff.mean()
