@@ -18,13 +18,22 @@
 //                supplies latent columns [256c + 128r, +128) of both pages.
 // Every CTA loads only its own tiles, from its own GPU's HBM, with plain (non-multicast) TMA.
 //
-// Warp roles (192 threads per CTA): warps 0-3 softmax + epilogue (thread i owns TMEM lane i:
-// head i % 64, token half i / 64), warp 4 TMA producer, warp 5 MMA issuer (leader CTA only) and
-// TMEM allocator.  Pipelines: a 7-slot ring of 16 KiB shared-memory slots for K and V tiles,
-// two S buffers in TMEM and two P buffers in shared memory, so QK^T of step g+1 runs while the
-// softmax of step g works.  The softmax rescales O only when a row max grows by more than 2^8
-// (exact after the final division by l).  Every wait is bounded: on timeout the kernel records
-// MLA_ERR_TIMEOUT, stops issuing work, and still frees its tensor memory before returning.
+// Warp roles (384 threads per CTA): warps 0-7 softmax + epilogue (two warps per TMEM lane
+// quadrant, each taking half of a lane's columns), warp 8 producer of Q and of the K ring,
+// warp 10 producer of the V ring, warp 9 QK^T issuer (leader CTA only) and TMEM allocator,
+// warp 11 PV issuer (leader CTA only).  Shared memory holds Q
+// (72 KiB), a K ring of three 24 KiB slots (one step: the CTA's page x 576 columns as three
+// groups of three 64-column blocks), a V ring of two 32 KiB slots (one per page of the step:
+// this CTA's 256 latent columns) and one P tile.  Tiles move as few, large TMA boxes (3-D and
+// 4-D views of the [rows, 576] cache whose inner dimensions are 64-column blocks): a single
+// thread issuing one small box at a time cannot reach HBM bandwidth, while one instruction per
+// 24-32 KiB can.  K and V have separate rings and producers, so a V slot held until its PV
+// never stalls the next step's K loads; the K producer also prefetches its pages into L2 three
+// steps ahead, so the shared-memory loads of a step see L2 rather than DRAM latency.  S is double-buffered in TMEM, so
+// QK^T of step g+1 runs while the softmax of step g works.  The softmax rescales O only when a
+// row max grows by more than 2^8 (exact after the final division by l).  Every wait is bounded:
+// on timeout the kernel records MLA_ERR_TIMEOUT, stops issuing work, and still frees its
+// tensor memory before returning.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -35,33 +44,41 @@ namespace mla {
 namespace {
 
 constexpr int H = 128, DROW = 576, PAGE = 64, STEP = 128;
-constexpr int NSLOT = 7;
-constexpr uint32_t BOX = 8192;                 // 64 rows x 128 bytes
-constexpr uint32_t SLOT = 2 * BOX;
+constexpr int NK = 3;                          // K ring: three slots of three 64-column blocks
+constexpr int NV = 2;                          // V ring: one slot per page of the step
+constexpr int PREFETCH_STEPS = 0;              // L2 prefetch distance of the K producer
+constexpr uint32_t BOX = 8192;                 // one 64-column block of 64 rows: 64 x 128 bytes
+constexpr uint32_t KSLOT = 3 * BOX;
+constexpr uint32_t VSLOT = 4 * BOX;            // [chunk 0..1][block pair][64 rows][64 cols]
 constexpr uint32_t Q_BYTES = 9 * BOX;          // 64 heads x 576 bf16
 constexpr uint32_t P_BYTES = 2 * BOX;          // 64 heads x 128 tokens bf16
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_P = OFF_Q + Q_BYTES;
-constexpr uint32_t OFF_SLOT = OFF_P + 2 * P_BYTES;
-constexpr uint32_t OFF_BAR = OFF_SLOT + NSLOT * SLOT;
+constexpr uint32_t OFF_K = OFF_P + P_BYTES;
+constexpr uint32_t OFF_V = OFF_K + NK * KSLOT;
+constexpr uint32_t OFF_BAR = OFF_V + NV * VSLOT;
 enum {
-    B_FULL = 0,
-    B_EMPTY = B_FULL + NSLOT,
-    B_QFULL = B_EMPTY + NSLOT,
+    B_KFULL = 0,
+    B_KEMPTY = B_KFULL + NK,
+    B_VFULL = B_KEMPTY + NK,
+    B_VEMPTY = B_VFULL + NV,
+    B_QFULL = B_VEMPTY + NV,
     B_QEMPTY,
     B_SFULL,
     B_SFREE = B_SFULL + 2,
     B_PFULL = B_SFREE + 2,
-    B_PVDONE = B_PFULL + 2,
+    B_PVDONE,
     B_OFREE = B_PVDONE + 2,
-    B_RED,                       // two barriers for the cross-warp exchange of row max / sum
-    B_COUNT = B_RED + 2
+    B_COUNT
 };
 constexpr uint32_t OFF_TMEMPTR = OFF_BAR + B_COUNT * 8;
 constexpr uint32_t OFF_FLAG = OFF_TMEMPTR + 8;
-constexpr uint32_t OFF_RED = (OFF_FLAG + 8 + 15) & ~15u;   // float[2][128]
-constexpr uint32_t SMEM_USED = OFF_RED + 2 * 128 * 4;
-constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;            // slack for 1024-byte alignment
+constexpr uint32_t OFF_RED = (OFF_FLAG + 8 + 15) & ~15u;   // float[2][2][128]
+constexpr uint32_t SMEM_USED = OFF_RED + 2 * 256 * 4;
+// The dynamic shared memory window starts 1024-byte aligned on sm_100 (the kernel checks this
+// and reports MLA_ERR_UNSUPPORTED instead of running if it ever does not).
+constexpr uint32_t SMEM_ALLOC = SMEM_USED;
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 constexpr uint32_t TM_S = 0;      // two S buffers of 64 columns
 constexpr uint32_t TM_O = 128;    // O: 256 columns
@@ -70,7 +87,11 @@ constexpr uint32_t TM_COLS = 512;
 constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(128, 256, false, true);
 constexpr uint64_t WAIT_NS = 2000000000ull;   // 2 s: no legitimate wait comes near this
-constexpr int SOFTMAX_WARPS = 4;
+constexpr int SOFTMAX_WARPS = 8;
+constexpr int SM_THREADS = 32 * SOFTMAX_WARPS;
+constexpr int W_KPROD = SOFTMAX_WARPS, W_MMA = SOFTMAX_WARPS + 1, W_VPROD = SOFTMAX_WARPS + 2,
+              W_PV = SOFTMAX_WARPS + 3;
+constexpr int THREADS = 32 * (SOFTMAX_WARPS + 4);
 constexpr float RESCALE_LOG2 = 8.f;           // rescale O when a row max grows by more than 2^8
 
 struct TcParams {
@@ -90,7 +111,8 @@ struct Ctx {
     volatile int *abort_flag;
     __device__ uint32_t bar(int i) const { return base + OFF_BAR + 8u * i; }
     __device__ uint32_t lead_bar(int i) const { return tc::map_to_rank(bar(i), 0); }
-    __device__ uint32_t slot(int s) const { return base + OFF_SLOT + SLOT * s; }
+    __device__ uint32_t kslot(int i) const { return base + OFF_K + KSLOT * i; }
+    __device__ uint32_t vslot(int i) const { return base + OFF_V + VSLOT * i; }
 };
 
 __device__ __forceinline__ bool wait_or_abort(const Ctx &c, uint32_t bar, uint32_t parity, int *err) {
@@ -119,95 +141,76 @@ __device__ __forceinline__ int page_row(const TcParams &p, int b, int pi, int t_
     return pid * PAGE;
 }
 
-// --------------------------------------------------------------------------- producer
-__device__ void run_producer(const Ctx &c, const TcParams &p, const CUtensorMap *tm_q, const CUtensorMap *tm_kv,
-                             int pair, int n_pairs) {
-    uint32_t u = 0;
-    int item_n = 0;
-    auto fill = [&](int nbox, int x0, int x1, int y) -> bool {
-        const int s = (int)(u % NSLOT);
-        const uint32_t use = u / NSLOT;
-        if (!wait_or_abort(c, c.bar(B_EMPTY + s), (use & 1u) ^ 1u, p.err)) return false;
-        const uint32_t full = c.lead_bar(B_FULL + s);
-        if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_FULL + s), 2u * nbox * BOX);
-        tc::tma_load_2d_pair(c.slot(s), tm_kv, x0, y, full);
-        if (nbox == 2) tc::tma_load_2d_pair(c.slot(s) + BOX, tm_kv, x1, y, full);
-        ++u;
-        return true;
-    };
-    auto fill_v = [&](int b, int t_step, int t_end) -> bool {
-        for (int ch = 0; ch < 2; ++ch)
-            for (int pg = 0; pg < 2; ++pg) {
-                const int y = page_row(p, b, t_step / PAGE + pg, t_end);
-                const int x = 256 * ch + 128 * (int)c.rank;
-                if (!fill(2, x, x + 64, y)) return false;
-            }
-        return true;
-    };
+// --------------------------------------------------------------------------- producers
+// Tensor maps (all over row-major [rows, 576] bf16 with 128-byte swizzle; the inner dimension is
+// one 64-column block, the row dimension has stride 1152 B, the block dimension stride 128 B):
+//   tm_q    3-D (64, rows, 9),    box (64, 64, 9): 64 rows x 576 columns, block-major in smem
+//   tm_k    3-D (64, rows, 9),    box (64, 64, 3): 64 rows x three blocks
+//   tm_page same map with box (64, 64, 9), used for the L2 prefetch of a whole page
+//   tm_v    4-D (64, rows, 4, 2), strides (1152, 128, 512), box (64, 64, 2, 2): for chunk c in
+//           {0, 1} the two blocks starting at 4c + 2 rank, i.e. columns [256c + 128 rank, +128)
+// K producer: per work item the CTA's 64 query heads (Q), then per 128-token step the CTA's own
+// page of the step.  Steps are numbered across items (g), so every slot's phase is g's parity.
+__device__ void run_k_producer(const Ctx &c, const TcParams &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                               const CUtensorMap *tm_page, int pair, int n_pairs) {
+    int g = 0, item_n = 0;
     for (int k = pair; k < p.plan.n_work; k += n_pairs) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) continue;   // only in a rejected plan, and then for every item
         const int b = it.row / p.s_q;
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
+        auto own_row = [&](int i) { return page_row(p, b, (it.t0 + STEP * i) / PAGE + (int)c.rank, it.t1); };
+        auto prefetch = [&](int i) {
+            const int y = own_row(i);
+            if (y < p.n_pages * PAGE) tc::tma_prefetch_3d(tm_page, 0, y, 0);
+        };
+        for (int i = 0; i < PREFETCH_STEPS && i < n_steps; ++i) prefetch(i);
         if (item_n > 0 && !wait_or_abort(c, c.bar(B_QEMPTY), (uint32_t)(item_n - 1) & 1u, p.err)) return;
         ++item_n;
         if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_QFULL), 2u * Q_BYTES);
-        const uint32_t qfull = c.lead_bar(B_QFULL);
-        const int qrow = it.row * H + 64 * (int)c.rank;
-        for (int cb = 0; cb < 9; ++cb) tc::tma_load_2d_pair(c.base + OFF_Q + cb * BOX, tm_q, 64 * cb, qrow, qfull);
-        for (int i = 0; i <= n_steps; ++i) {
-            if (i < n_steps) {
-                const int t_step = it.t0 + STEP * i;
-                const int y = page_row(p, b, t_step / PAGE + (int)c.rank, it.t1);
-                for (int j = 0; j < 4; ++j)
-                    if (!fill(2, 128 * j, 128 * j + 64, y)) return;
-                if (!fill(1, 512, 0, y)) return;
+        tc::tma_load_3d_pair(c.base + OFF_Q, tm_q, 0, it.row * H + 64 * (int)c.rank, 0, c.lead_bar(B_QFULL));
+        for (int i = 0; i < n_steps; ++i, ++g) {
+            if (i + PREFETCH_STEPS < n_steps) prefetch(i + PREFETCH_STEPS);
+            const int y = own_row(i);
+            for (int j = 0; j < NK; ++j) {
+                if (!wait_or_abort(c, c.bar(B_KEMPTY + j), ((uint32_t)g & 1u) ^ 1u, p.err)) return;
+                if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_KFULL + j), 2u * KSLOT);
+                tc::tma_load_3d_pair(c.kslot(j), tm_k, 0, y, 3 * j, c.lead_bar(B_KFULL + j));
             }
-            if (i >= 1 && !fill_v(b, it.t0 + STEP * (i - 1), it.t1)) return;
         }
     }
 }
 
-// --------------------------------------------------------------------------- MMA issuer
-__device__ void run_mma(const Ctx &c, const TcParams &p, uint32_t tmem, int pair, int n_pairs) {
-    uint32_t u = 0;
-    int g = 0, item_n = 0;
-    auto take = [&](int &s) -> bool {
-        s = (int)(u % NSLOT);
-        const uint32_t use = u / NSLOT;
-        ++u;
-        if (!wait_or_abort(c, c.bar(B_FULL + s), use & 1u, p.err)) return false;
-        tc::fence_after_sync();
-        return true;
-    };
-    auto pv = [&](int gj, bool first) -> bool {
-        const int pb = gj & 1;
-        if (!wait_or_abort(c, c.bar(B_PFULL + pb), (uint32_t)(gj >> 1) & 1u, p.err)) return false;
-        if (first && item_n > 0 && !wait_or_abort(c, c.bar(B_OFREE), (uint32_t)(item_n - 1) & 1u, p.err))
-            return false;
-        tc::fence_after_sync();
-        const uint32_t pbase = c.base + OFF_P + P_BYTES * pb;
-        for (int ch = 0; ch < 2; ++ch)
-            for (int pg = 0; pg < 2; ++pg) {
-                int s;
-                if (!take(s)) return false;
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const uint64_t a = tc::sdesc_sw128(pbase + pg * BOX + 32 * k4, 16, 1024);
-                    const uint64_t bd = tc::sdesc_sw128(c.slot(s) + 2048 * k4, BOX, 1024);
-                    tc::mma_pair_bf16(tmem + TM_O + 128 * ch, a, bd, IDESC_PV, (first && pg == 0 && k4 == 0) ? 0u : 1u);
-                }
-                tc::commit_pair(c.bar(B_EMPTY + s), 0x3);
-            }
-        tc::commit_pair(c.bar(B_PVDONE + pb), 0x3);
-        return true;
-    };
-    for (int k = pair; k < p.plan.n_work; k += n_pairs, ++item_n) {
+// V producer: per step and page pg of the step, this CTA's 256 latent columns of that page.
+__device__ void run_v_producer(const Ctx &c, const TcParams &p, const CUtensorMap *tm_v, int pair, int n_pairs) {
+    int g = 0;
+    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
         const WorkItem it = p.plan.items[k];
-        if (it.t1 <= it.t0) {
-            --item_n;   // only in a rejected plan, and then for every item
-            continue;
+        if (it.t1 <= it.t0) continue;
+        const int b = it.row / p.s_q;
+        const int n_steps = ceil_div(it.t1 - it.t0, STEP);
+        for (int i = 0; i < n_steps; ++i, ++g) {
+            const int t_step = it.t0 + STEP * i;
+            for (int pg = 0; pg < NV; ++pg) {
+                const int y = page_row(p, b, t_step / PAGE + pg, it.t1);
+                if (!wait_or_abort(c, c.bar(B_VEMPTY + pg), ((uint32_t)g & 1u) ^ 1u, p.err)) return;
+                if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_VFULL + pg), 2u * VSLOT);
+                tc::tma_load_4d_pair(c.vslot(pg), tm_v, 0, y, 2 * (int)c.rank, 0, c.lead_bar(B_VFULL + pg));
+            }
         }
+    }
+}
+
+// --------------------------------------------------------------------------- MMA issuers
+// Two threads of the leader CTA issue the pair's MMAs, each waiting only on its own inputs, so
+// the in-order tensor pipe always has whichever of QK^T(g + 1) and PV(g) is ready.  A
+// tcgen05.commit tracks the MMAs of the thread that issues it, so each issuer's barriers
+// report exactly its own work.
+__device__ void run_qk_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, int pair, int n_pairs) {
+    int g = 0, item_n = 0;
+    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
+        const WorkItem it = p.plan.items[k];
+        if (it.t1 <= it.t0) continue;   // only in a rejected plan, and then for every item
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
         if (!wait_or_abort(c, c.bar(B_QFULL), (uint32_t)item_n & 1u, p.err)) return;
         tc::fence_after_sync();
@@ -216,53 +219,87 @@ __device__ void run_mma(const Ctx &c, const TcParams &p, uint32_t tmem, int pair
             if (g >= 2 && !wait_or_abort(c, c.bar(B_SFREE + sb), (uint32_t)((g - 2) >> 1) & 1u, p.err)) return;
             tc::fence_after_sync();
             const uint32_t d = tmem + TM_S + 64 * sb;
-            for (int j = 0; j < 5; ++j) {
-                int s;
-                if (!take(s)) return;
-                const int nk = j < 4 ? 8 : 4;
-                for (int kk = 0; kk < nk; ++kk) {
-                    const int cb = 2 * j + kk / 4, w4 = kk % 4;
-                    const uint64_t a = tc::sdesc_sw128(c.base + OFF_Q + cb * BOX + 32 * w4, 16, 1024);
-                    const uint64_t bd = tc::sdesc_sw128(c.slot(s) + (kk / 4) * BOX + 32 * w4, 16, 1024);
-                    tc::mma_pair_bf16(d, a, bd, IDESC_QK, (j | kk) ? 1u : 0u);
+            for (int j = 0; j < NK; ++j) {
+                if (!wait_or_abort(c, c.bar(B_KFULL + j), (uint32_t)g & 1u, p.err)) return;
+                tc::fence_after_sync();
+                for (int q3 = 0; q3 < 3; ++q3) {
+                    const int cb = 3 * j + q3;
+#pragma unroll
+                    for (int w4 = 0; w4 < 4; ++w4) {
+                        const uint64_t a = tc::sdesc_sw128(c.base + OFF_Q + cb * BOX + 32 * w4, 16, 1024);
+                        const uint64_t bd = tc::sdesc_sw128(c.kslot(j) + q3 * BOX + 32 * w4, 16, 1024);
+                        tc::mma_pair_bf16(d, a, bd, IDESC_QK, (cb | w4) ? 1u : 0u);
+                    }
                 }
-                tc::commit_pair(c.bar(B_EMPTY + s), 0x3);
+                tc::commit_pair(c.bar(B_KEMPTY + j), 0x3);
             }
             if (i == n_steps - 1) tc::commit_pair(c.bar(B_QEMPTY), 0x3);
             tc::commit_pair(c.bar(B_SFULL + sb), 0x3);
-            if (i >= 1 && !pv(g - 1, i == 1)) return;
         }
-        if (!pv(g - 1, n_steps == 1)) return;
+        ++item_n;
+    }
+}
+
+__device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, int pair, int n_pairs) {
+    int g = 0, item_n = 0;
+    const uint32_t pbase = c.base + OFF_P;
+    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
+        const WorkItem it = p.plan.items[k];
+        if (it.t1 <= it.t0) continue;
+        const int n_steps = ceil_div(it.t1 - it.t0, STEP);
+        for (int i = 0; i < n_steps; ++i, ++g) {
+            if (!wait_or_abort(c, c.bar(B_PFULL), (uint32_t)g & 1u, p.err)) return;
+            // The first PV of an item overwrites O: the previous item's epilogue must be done with it.
+            if (i == 0 && item_n > 0 && !wait_or_abort(c, c.bar(B_OFREE), (uint32_t)(item_n - 1) & 1u, p.err)) return;
+            tc::fence_after_sync();
+            for (int pg = 0; pg < NV; ++pg) {
+                if (!wait_or_abort(c, c.bar(B_VFULL + pg), (uint32_t)g & 1u, p.err)) return;
+                tc::fence_after_sync();
+                for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const uint64_t a = tc::sdesc_sw128(pbase + pg * BOX + 32 * k4, 16, 1024);
+                        const uint64_t bd = tc::sdesc_sw128(c.vslot(pg) + 2 * BOX * ch + 2048 * k4, BOX, 1024);
+                        tc::mma_pair_bf16(tmem + TM_O + 128 * ch, a, bd, IDESC_PV, (i == 0 && pg == 0 && k4 == 0) ? 0u : 1u);
+                    }
+                }
+                tc::commit_pair(c.bar(B_VEMPTY + pg), 0x3);
+            }
+            tc::commit_pair(c.bar(B_PVDONE + (g & 1)), 0x3);
+        }
+        ++item_n;
     }
 }
 
 // --------------------------------------------------------------------------- softmax + epilogue
+// Eight warps, two per TMEM lane quadrant: warp w reads lanes [32 (w % 4), +32) and column half
+// w / 4 of each S buffer, so thread t owns lane L = 32 (w % 4) + lane, i.e. head L % 64, tokens
+// 64 (L / 64) + 32 (w / 4) + [0, 32) of the step.  The four threads of a head swap their maxima
+// and, at the end, their sums through shared memory behind a named barrier.  Control flow does
+// not depend on data or on a wait's outcome: a wait that runs out only records the error, so
+// every thread always reaches every named barrier.
 __device__ void run_softmax(const Ctx &c, const TcParams &p, uint32_t tmem, int pair, int n_pairs) {
-    const int L = threadIdx.x;  // TMEM lane, 0..127
-    const int warp = L / 32, lane = L % 32;
+    const int t = threadIdx.x;                     // 0..255
+    const int warp = t / 32, lane = t % 32;
+    const int quad = warp & 3, half = warp >> 2;
+    const int L = 32 * quad + lane;                // TMEM lane
     const int hl = L & 63, hsel = L >> 6;
     const int head = 64 * (int)c.rank + hl;
-    const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
-    float *red = reinterpret_cast<float *>(c.sbase + OFF_RED);
-    int g = 0, item_n = 0;
-    bool ok = true;
-    // The two threads of a head (TMEM lanes L and L ^ 64) sit in different warps; they swap a
-    // value through shared memory behind a 128-arrival mbarrier (bounded wait, no bar.sync that
-    // could outlive an aborted warp).  Exchange x uses buffer x % 2.
-    uint32_t xchg = 0;
-    auto exchange = [&](float v, float &other) -> bool {
-        const int bi = (int)(xchg & 1u);
-        red[128 * bi + L] = v;
-        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(c.bar(B_RED + bi)) : "memory");
-        const bool w = warp_wait(c, c.bar(B_RED + bi), (xchg >> 1) & 1u, p.err);
-        if (w) other = red[128 * bi + (L ^ 64)];
-        ++xchg;
-        return w;
+    const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
+    float *red = reinterpret_cast<float *>(c.sbase + OFF_RED);   // [2][2][128]
+    auto others = [&](int buf, float v, float &a, float &b, float &d) {
+        float *r = red + 256 * buf;
+        r[128 * half + L] = v;
+        tc::named_sync(1, SM_THREADS);
+        a = r[128 * (half ^ 1) + L];
+        b = r[128 * half + (L ^ 64)];
+        d = r[128 * (half ^ 1) + (L ^ 64)];
     };
-    for (int k = pair; k < p.plan.n_work && ok; k += n_pairs, ++item_n) {
+    int g = 0;
+    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) {
-            if (hsel == 0) {
+            if (hsel == 0 && half == 0) {
                 p.part_ml[((size_t)k * H + head) * 2] = -INFINITY;
                 p.part_ml[((size_t)k * H + head) * 2 + 1] = 0.f;
             }
@@ -272,100 +309,104 @@ __device__ void run_softmax(const Ctx &c, const TcParams &p, uint32_t tmem, int 
         float m_run = -INFINITY, l_run = 0.f;
         for (int i = 0; i < n_steps; ++i, ++g) {
             const int sb = g & 1;
-            if (!(ok = warp_wait(c, c.bar(B_SFULL + sb), (uint32_t)(g >> 1) & 1u, p.err))) break;
+            warp_wait(c, c.bar(B_SFULL + sb), (uint32_t)(g >> 1) & 1u, p.err);
             tc::fence_after_sync();
-            float s[64];
-            tc::tmem_ld64(tmem + TM_S + 64 * sb + lane_addr, s);
+            float s[32];
+            tc::tmem_ld32(tmem + TM_S + 64 * sb + 32 * half + lane_addr, s);
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive_cluster(c.lead_bar(B_SFREE + sb));
 
-            const int tok0 = it.t0 + STEP * i + 64 * hsel;
-            const int nvalid = min(64, max(0, it.t1 - tok0));
-            float mx = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                s[j] = j < nvalid ? s[j] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[j]);
-            }
-            float mo = -INFINITY;
-            if (!(ok = exchange(mx, mo))) break;
-            const float mt = fmaxf(mx, mo);
-            if (i == 0 || mt > m_run + RESCALE_LOG2) {
-                if (i > 0) {
-                    const float alpha = exp2f(m_run - mt);
-                    // O holds steps < g: wait until PV(g-1) has landed, then rescale in place.
-                    if (!(ok = warp_wait(c, c.bar(B_PVDONE + ((g - 1) & 1)), (uint32_t)((g - 1) >> 1) & 1u, p.err)))
-                        break;
-                    tc::fence_after_sync();
-#pragma unroll 1
-                    for (int q = 0; q < 4; ++q) {
-                        float v[64];
-                        tc::tmem_ld64(tmem + TM_O + 64 * q + lane_addr, v);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 64; ++j) v[j] *= alpha;
-                        tc::tmem_st64(tmem + TM_O + 64 * q + lane_addr, v);
-                    }
-                    tc::tmem_wait_st();
-                    l_run *= alpha;
-                }
-                m_run = mt;
-            }
-            float sum = 0.f;
-            uint32_t pk[32];
+            const int tok0 = it.t0 + STEP * i + 64 * hsel + 32 * half;
+            const int nvalid = min(32, max(0, it.t1 - tok0));
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                const float a = exp2f(s[2 * j] - m_run), b2 = exp2f(s[2 * j + 1] - m_run);
-                sum += a + b2;
+                s[j] = j < nvalid ? s[j] : -INFINITY;
+                m4[j & 3] = fmaxf(m4[j & 3], s[j]);
+            }
+            float o1, o2, o3;
+            others(g & 1, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])), o1, o2, o3);
+            const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            const float m_tile = fmaxf(fmaxf(mt, o1), fmaxf(o2, o3)) * p.scale_log2;   // head max, log2 units
+            // One rescale decision for all heads keeps the tcgen05 loads below warp-uniform.
+            const bool any = tc::named_sync_or(2, SM_THREADS, i > 0 && m_tile > m_run + RESCALE_LOG2);
+            // PV(g-1) must be complete before O is rescaled and before P is overwritten.
+            if (g >= 1) warp_wait(c, c.bar(B_PVDONE + ((g - 1) & 1)), (uint32_t)((g - 1) >> 1) & 1u, p.err);
+            tc::fence_after_sync();
+            if (i == 0) {
+                m_run = m_tile;
+            } else if (any) {
+                const float m_new = fmaxf(m_run, m_tile);
+                const float alpha = tc::ex2(m_run - m_new);
+#pragma unroll 1
+                for (int q = 0; q < 2; ++q) {
+                    float v[64];
+                    const uint32_t a = tmem + TM_O + 128 * half + 64 * q + lane_addr;
+                    tc::tmem_ld64(a, v);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) v[j] *= alpha;
+                    tc::tmem_st64(a, v);
+                }
+                tc::tmem_wait_st();
+                l_run *= alpha;
+                m_run = m_new;
+            }
+            const float neg_m = -m_run;
+            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float a = tc::ex2(fmaf(s[2 * j], p.scale_log2, neg_m));
+                const float b2 = tc::ex2(fmaf(s[2 * j + 1], p.scale_log2, neg_m));
+                sum4[j & 3] += a + b2;
                 __nv_bfloat162 h2 = __floats2bfloat162_rn(a, b2);
                 pk[j] = *reinterpret_cast<uint32_t *>(&h2);
             }
-            l_run += sum;
-            // P buffer g%2 was read by PV(g-2).
-            if (g >= 2 && !(ok = warp_wait(c, c.bar(B_PVDONE + sb), (uint32_t)((g - 2) >> 1) & 1u, p.err))) break;
-            uint8_t *prow = c.sbase + OFF_P + P_BYTES * sb + BOX * hsel + 128 * hl;
+            l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+            uint8_t *prow = c.sbase + OFF_P + BOX * hsel + 128 * hl;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-                *reinterpret_cast<uint4 *>(prow + ((ch ^ (hl & 7)) << 4)) = v;
+            for (int ch = 0; ch < 4; ++ch) {
+                const uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+                *reinterpret_cast<uint4 *>(prow + (((4 * half + ch) ^ (hl & 7)) << 4)) = v;
             }
             tc::fence_proxy_async_smem();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive_cluster(c.lead_bar(B_PFULL + sb));
+            if (lane == 0) tc::mbar_arrive_cluster(c.lead_bar(B_PFULL));
         }
-        if (!ok) break;
         // Epilogue: the last PV of this item has landed; write the partial O, m, l.
-        if (!(ok = warp_wait(c, c.bar(B_PVDONE + ((g - 1) & 1)), (uint32_t)((g - 1) >> 1) & 1u, p.err))) break;
+        warp_wait(c, c.bar(B_PVDONE + ((g - 1) & 1)), (uint32_t)((g - 1) >> 1) & 1u, p.err);
         tc::fence_after_sync();
-        float lo = 0.f;
-        if (!(ok = exchange(l_run, lo))) break;
-        const float l_tot = l_run + lo;
-        float *dst = p.part_o + ((size_t)k * H + head) * 512;
+        float l1, l2, l3;
+        others(g & 1, l_run, l1, l2, l3);
+        const float l_tot = (l_run + l1) + (l2 + l3);
+        float *dst = p.part_o + ((size_t)k * H + head) * 512 + 256 * half + 128 * hsel;
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
             float v[64];
-            tc::tmem_ld64(tmem + TM_O + 64 * q + lane_addr, v);
+            tc::tmem_ld64(tmem + TM_O + 128 * half + 64 * q + lane_addr, v);
             tc::tmem_wait_ld();
-            const int d0 = 256 * (q / 2) + 128 * hsel + 64 * (q % 2);
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-                *reinterpret_cast<float4 *>(dst + d0 + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                *reinterpret_cast<float4 *>(dst + 64 * q + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         }
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive_cluster(c.lead_bar(B_OFREE));
-        if (hsel == 0) {
+        if (hsel == 0 && half == 0) {
             p.part_ml[((size_t)k * H + head) * 2] = m_run * 0.69314718055994531f;
             p.part_ml[((size_t)k * H + head) * 2 + 1] = l_tot;
         }
+        tc::named_sync(1, SM_THREADS);   // the next item's first exchange reuses buffer g & 1
     }
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-    tc_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv, TcParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    tc_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_page, const __grid_constant__ CUtensorMap tm_v, TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     Ctx c;
     const uint32_t raw = tc::smem_addr(smem_raw);
@@ -374,31 +415,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     c.rank = tc::cluster_rank();
     c.abort_flag = reinterpret_cast<volatile int *>(c.sbase + OFF_FLAG);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    uint32_t dyn_bytes;
+    asm("mov.u32 %0, %dynamic_smem_size;" : "=r"(dyn_bytes));
+    if (c.base - raw + SMEM_USED > dyn_bytes) {   // uniform for the whole cluster: nothing ran yet
+        if (threadIdx.x == 0) report(p.err, MLA_ERR_UNSUPPORTED);
+        return;
+    }
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NSLOT; ++i) {
-            tc::mbar_init(c.bar(B_FULL + i), 1);
-            tc::mbar_init(c.bar(B_EMPTY + i), 1);
+        for (int i = 0; i < NK; ++i) {
+            tc::mbar_init(c.bar(B_KFULL + i), 1);
+            tc::mbar_init(c.bar(B_KEMPTY + i), 1);
+        }
+        for (int i = 0; i < NV; ++i) {
+            tc::mbar_init(c.bar(B_VFULL + i), 1);
+            tc::mbar_init(c.bar(B_VEMPTY + i), 1);
         }
         tc::mbar_init(c.bar(B_QFULL), 1);
         tc::mbar_init(c.bar(B_QEMPTY), 1);
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(c.bar(B_SFULL + i), 1);
             tc::mbar_init(c.bar(B_SFREE + i), 2 * SOFTMAX_WARPS);
-            tc::mbar_init(c.bar(B_PFULL + i), 2 * SOFTMAX_WARPS);
             tc::mbar_init(c.bar(B_PVDONE + i), 1);
         }
+        tc::mbar_init(c.bar(B_PFULL), 2 * SOFTMAX_WARPS);
         tc::mbar_init(c.bar(B_OFREE), 2 * SOFTMAX_WARPS);
-        tc::mbar_init(c.bar(B_RED), 32 * SOFTMAX_WARPS);
-        tc::mbar_init(c.bar(B_RED + 1), 32 * SOFTMAX_WARPS);
         *c.abort_flag = 0;
         tc::fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == W_KPROD && lane == 0) {
         tc::prefetch_tmap(&tm_q);
-        tc::prefetch_tmap(&tm_kv);
+        tc::prefetch_tmap(&tm_k);
+        tc::prefetch_tmap(&tm_page);
+        tc::prefetch_tmap(&tm_v);
     }
-    if (warp == 5) tc::tmem_alloc_pair(c.base + OFF_TMEMPTR, TM_COLS);
+    if (warp == W_MMA) tc::tmem_alloc_pair(c.base + OFF_TMEMPTR, TM_COLS);
     tc::fence_before_sync();
     __syncthreads();
     tc::cluster_sync();
@@ -406,10 +457,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(c.sbase + OFF_TMEMPTR);
 
     const int pair = blockIdx.x / 2, n_pairs = gridDim.x / 2;
-    if (warp == 4) {
-        if (lane == 0) run_producer(c, p, &tm_q, &tm_kv, pair, n_pairs);
-    } else if (warp == 5) {
-        if (c.rank == 0 && lane == 0) run_mma(c, p, tmem, pair, n_pairs);
+    if (warp == W_KPROD) {
+        if (lane == 0) run_k_producer(c, p, &tm_q, &tm_k, &tm_page, pair, n_pairs);
+    } else if (warp == W_VPROD) {
+        if (lane == 0) run_v_producer(c, p, &tm_v, pair, n_pairs);
+    } else if (warp == W_MMA) {
+        if (c.rank == 0 && lane == 0) run_qk_issuer(c, p, tmem, pair, n_pairs);
+    } else if (warp == W_PV) {
+        if (c.rank == 0 && lane == 0) run_pv_issuer(c, p, tmem, pair, n_pairs);
     } else {
         run_softmax(c, p, tmem, pair, n_pairs);
     }
@@ -424,7 +479,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::cluster_sync();
-    if (warp == 5) {
+    if (warp == W_MMA) {
         tc::fence_after_sync();
         tc::tmem_dealloc_pair(tmem, TM_COLS);
         tc::tmem_relinquish_pair();
@@ -447,15 +502,26 @@ EncodeTiled encode_fn() {
     return fn;
 }
 
-// [rows, 576] bf16 row-major, 64x64 boxes with 128-byte swizzle (zero fill past the end).
-bool encode_rows576(CUtensorMap *m, const void *ptr, uint64_t rows) {
+// Views of a row-major [rows, 576] bf16 matrix whose innermost dimension is one 64-column
+// block (128 bytes, swizzled), so one box gathers several blocks of 64 rows block-major into
+// shared memory.  `nblk` = blocks per box; with `vsplit` the blocks are addressed as
+// [4 blocks per 256-column chunk][2 chunks].  Zero fill past the end.
+bool encode_blocks(CUtensorMap *m, const void *ptr, uint64_t rows, int nblk, bool vsplit) {
     EncodeTiled fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {DROW, rows};
-    cuuint64_t strides[1] = {DROW * 2};
-    cuuint32_t box[2] = {64, 64};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (!vsplit) {
+        cuuint64_t dims[3] = {64, rows, 9};
+        cuuint64_t strides[2] = {DROW * 2, 128};
+        cuuint32_t box[3] = {64, 64, (cuuint32_t)nblk};
+        return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
+    cuuint64_t dims[4] = {64, rows, 4, 2};
+    cuuint64_t strides[3] = {DROW * 2, 128, 512};
+    cuuint32_t box[4] = {64, 64, 2, 2};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -470,9 +536,11 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
                              const Plan &plan, int max_pages, int n_pages, int s_q, float *part_o, float *part_ml,
                              int *err, int sms, cudaStream_t st) {
     if (plan.n_work == 0) return cudaSuccess;
-    CUtensorMap tm_q, tm_kv;
-    if (!encode_rows576(&tm_q, q_abs, (uint64_t)plan.rows * H) ||
-        !encode_rows576(&tm_kv, latent, (uint64_t)n_pages * PAGE))
+    CUtensorMap tm_q, tm_k, tm_page, tm_v;
+    const uint64_t kv_rows = (uint64_t)n_pages * PAGE;
+    if (!encode_blocks(&tm_q, q_abs, (uint64_t)plan.rows * H, 9, false) ||
+        !encode_blocks(&tm_k, latent, kv_rows, 3, false) || !encode_blocks(&tm_page, latent, kv_rows, 9, false) ||
+        !encode_blocks(&tm_v, latent, kv_rows, 0, true))
         return cudaErrorInvalidValue;
     TcParams p;
     p.plan = plan;
@@ -491,7 +559,7 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
         attr_set = true;
     }
     const int units = std::max(1, std::min(plan.n_work, std::max(1, sms / 2)));
-    tc_decode_kernel<<<2 * units, 192, SMEM_ALLOC, st>>>(tm_q, tm_kv, p);
+    tc_decode_kernel<<<2 * units, THREADS, SMEM_ALLOC, st>>>(tm_q, tm_k, tm_page, tm_v, p);
     return cudaGetLastError();
 }
 
