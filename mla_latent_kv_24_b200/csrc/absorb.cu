@@ -113,3 +113,105 @@ cudaError_t launch_q_rope(const Dims &d, const void *q, const int *seq_lens, int
 }
 
 }  // namespace mla
+
+// ---------------------------------------------------------------------------------------
+// Tensor-core q absorption for the DeepSeek-V2 shape (bf16, d_nope = 128, d_c = 512,
+// d_rope = 64).  Per head it is the GEMM q_lat[rows, 512] = q_nope[rows, 128] W_UK[w]
+// ([128, 512], row k = nope dim).  One CTA computes 64 query rows x 128 latent columns of one
+// head with mma.sync m16n8k16: the W_UK tile [128 k][64 n] and the q tile [64][128] are staged
+// in padded shared memory by cp.async, B fragments come through ldmatrix.trans.  Every W_UK
+// element is read once per head (16.8 MB in total for H = 128), the bound of this step.
+// CTAs of the first column tile also rotate the query's RoPE part.
+// ---------------------------------------------------------------------------------------
+#include "warp_mma.cuh"
+
+namespace mla {
+namespace {
+
+constexpr int AB_M = 64, AB_N = 64, AB_K = 128, AB_LD = AB_K + 8, AB_LDB = AB_N + 8;
+
+__global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                           const __nv_bfloat16 *__restrict__ W_uk,
+                                                           const int *__restrict__ seq_lens, int rows, int s_q,
+                                                           int H, int hpw, float base,
+                                                           __nv_bfloat16 *__restrict__ q_abs) {
+    __shared__ __align__(16) __nv_bfloat16 As[AB_M * AB_LD];    // [64 rows][128 k]
+    __shared__ __align__(16) __nv_bfloat16 Bs[AB_K * AB_LDB];   // [128 k][64 n]
+    const int h = blockIdx.x, n0 = blockIdx.y * AB_N, row0 = blockIdx.z * AB_M;
+    const int w = h / hpw, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    constexpr int D_C = 512, D_N = 128, D_R = 64, D_QK = 192, D_OUT = 576;
+    const __nv_bfloat16 *Wk = W_uk + (size_t)w * D_N * D_C;
+    for (int c = tid; c < AB_K * AB_N / 8; c += 256) {          // 2048 chunks of 16 B
+        const int k = c / (AB_N / 8), n = (c % (AB_N / 8)) * 8;
+        cp_async16(Bs + k * AB_LDB + n, Wk + (size_t)k * D_C + n0 + n, true);
+    }
+    for (int c = tid; c < AB_M * AB_K / 8; c += 256) {
+        const int r = c / (AB_K / 8), k = (c % (AB_K / 8)) * 8;
+        const int row = row0 + r;
+        cp_async16(As + r * AB_LD + k, q + ((size_t)(row < rows ? row : 0) * H + h) * D_QK + k, row < rows);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    // warp tile: 16 rows x 32 columns (4 n8 tiles); 4 x 2 warps cover 64 x 64
+    const int wm = warp % 4, wn = warp / 4;
+    float acc[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < AB_K; kk += 16) {
+        uint32_t a[4];
+        ldmatrix_x4(a[0], a[1], a[2], a[3],
+                    As + (wm * 16 + (lane % 8) + 8 * ((lane / 8) % 2)) * AB_LD + kk + 8 * (lane / 16));
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+            // B stored [k][n]: .trans gives the k-major fragments of two n8 tiles
+            uint32_t b0, b1, b2, b3;
+            const int kr = kk + (lane % 8) + 8 * ((lane / 8) % 2);
+            const int nc = wn * 32 + j * 8 + 8 * (lane / 16);
+            ldmatrix_x4_trans(b0, b1, b2, b3, Bs + kr * AB_LDB + nc);
+            mma_bf16(acc[j], a, b0, b1);
+            mma_bf16(acc[j + 1], a, b2, b3);
+        }
+    }
+    const int gid = lane / 4, t4 = lane % 4;
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+        const int row = row0 + wm * 16 + gid + 8 * hr;
+        if (row >= rows) continue;
+        __nv_bfloat16 *dst = q_abs + ((size_t)row * H + h) * D_OUT + n0 + wn * 32;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint32_t *>(dst + j * 8 + 2 * t4) = pack_bf16(acc[j][2 * hr], acc[j][2 * hr + 1]);
+    }
+    if (blockIdx.y == 0) {   // RoPE part of the query, rows of this tile
+        for (int i = tid; i < AB_M * (D_R / 2); i += 256) {
+            const int r = i / (D_R / 2), pi = i % (D_R / 2), row = row0 + r;
+            if (row >= rows) continue;
+            const int b = row / s_q, j = row % s_q, pos = seq_lens[b] - s_q + j;
+            const __nv_bfloat16 *src = q + ((size_t)row * H + h) * D_QK + D_N + 2 * pi;
+            float x0 = __bfloat162float(src[0]), x1 = __bfloat162float(src[1]), cs, sn;
+            rope_cos_sin(pos, pi, D_R, base, &cs, &sn);
+            __nv_bfloat16 *o = q_abs + ((size_t)row * H + h) * D_OUT + D_C + 2 * pi;
+            o[0] = __float2bfloat16_rn(x0 * cs - x1 * sn);
+            o[1] = __float2bfloat16_rn(x0 * sn + x1 * cs);
+        }
+    }
+}
+
+}  // namespace
+
+bool q_absorb_mma_ok(const Dims &d) { return d.bf16 && d.d_n == 128 && d.d_c == 512 && d.d_r == 64; }
+
+cudaError_t launch_q_absorb_mma(const Dims &d, const void *q, const void *W_uk, const int *seq_lens, int batch,
+                                int s_q, void *q_abs, cudaStream_t st) {
+    const int rows = batch * s_q;
+    dim3 grid(d.H, 512 / AB_N, ceil_div(rows, AB_M));
+    q_absorb_mma_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)W_uk, seq_lens, rows,
+                                              s_q, d.H, d.hpw, d.base, (__nv_bfloat16 *)q_abs);
+    return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -240,9 +240,14 @@ mla_status mla_cache_append(const mla_dims *dims, const void *h, int32_t hidden,
     if (batch <= 0 || max_pages <= 0 || n_pages_total <= 0) return fail(MLA_ERR_INVALID_ARG, "batch, max_pages, n_pages_total must be > 0");
     int *err = nullptr;
     MLA_TRY(device_info(&err, nullptr));
-    MLA_CUDA(launch_append(d, h, hidden, W_dkv, W_kr, req_idx, positions, n_tok, page_table, batch, max_pages,
-                           n_pages_total, latent_cache, err, (cudaStream_t)stream),
-             "launch cache_append");
+    if (append_mma_ok(d, hidden, W_dkv != nullptr) && aligned16(h) && aligned16(W_dkv) && aligned16(W_kr))
+        MLA_CUDA(launch_append_mma(d, h, hidden, W_dkv, W_kr, req_idx, positions, n_tok, page_table, batch, max_pages,
+                                   n_pages_total, latent_cache, err, (cudaStream_t)stream),
+                 "launch cache_append (tensor cores)");
+    else
+        MLA_CUDA(launch_append(d, h, hidden, W_dkv, W_kr, req_idx, positions, n_tok, page_table, batch, max_pages,
+                               n_pages_total, latent_cache, err, (cudaStream_t)stream),
+                 "launch cache_append");
     return MLA_OK;
 }
 
@@ -309,7 +314,10 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
     MLA_CUDA(launch_plan(seq_lens, batch, s_q, max_pages, d.page, L.chunk, L.n_work, items, row_first, err, st),
              "launch plan");
     if (path == ABSORBED) {
-        MLA_CUDA(launch_q_absorb(d, q, W_uk, seq_lens, batch, s_q, qp, st), "launch q_absorb");
+        if (q_absorb_mma_ok(d))
+            MLA_CUDA(launch_q_absorb_mma(d, q, W_uk, seq_lens, batch, s_q, qp, st), "launch q_absorb (tensor cores)");
+        else
+            MLA_CUDA(launch_q_absorb(d, q, W_uk, seq_lens, batch, s_q, qp, st), "launch q_absorb");
         if (tc) {
             ProfileScope prof(st);
             MLA_CUDA(launch_tc_decode(d, qp, latent, page_table, plan, max_pages, n_pages, s_q, part_o, part_ml, err, sms,
@@ -320,7 +328,11 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
             SimtDecodeArgs a{qp, latent, nullptr, page_table, plan, max_pages, n_pages, s_q, 0, part_o, part_ml, err};
             MLA_CUDA(launch_decode_simt(d, a, st), "launch decode (CUDA cores)");
         }
-        MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, L.DV, W_uv, out, st), "launch combine");
+        if (combine_mma_ok(d, L.DV, true))
+            MLA_CUDA(launch_combine_mma(d, part_o, part_ml, row_first, L.rows, W_uv, out, st),
+                     "launch combine + W_UV (tensor cores)");
+        else
+            MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, L.DV, W_uv, out, st), "launch combine");
     } else {
         if (grouped_tc_ok(d)) {
             ProfileScope prof(st);

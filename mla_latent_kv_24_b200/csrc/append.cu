@@ -111,3 +111,127 @@ cudaError_t launch_append(const Dims &d, const void *h, int hidden, const void *
 }
 
 }  // namespace mla
+
+// ---------------------------------------------------------------------------------------
+// Tensor-core append for the DeepSeek-V2 shape (bf16, d_c = 512, d_rope = 64, hidden a multiple
+// of 256 up to 10240).  The projection [n_tok, hidden] x [hidden, 576] is weight-bandwidth bound for a
+// decode batch (n_tok = batch * s_q), so the weights must stream through many SMs at once: a
+// cluster of 8 CTAs splits the hidden dimension, each CTA multiplies its slice of 16 tokens x
+// 64 output columns with mma.sync, and rank 0 sums the 8 partial tiles through distributed
+// shared memory, then applies RoPE and scatters into the paged cache.  Grid: 9 column tiles x 8
+// hidden slices (72 CTAs) per 16-token tile.
+// ---------------------------------------------------------------------------------------
+#include <cooperative_groups.h>
+
+#include "warp_mma.cuh"
+
+namespace mla {
+namespace {
+
+constexpr int AP_SPLIT = 8, AP_COLS = 64, AP_TOK = 16;
+
+__global__ void __cluster_dims__(AP_SPLIT, 1, 1) __launch_bounds__(256)
+    append_mma_kernel(const __nv_bfloat16 *__restrict__ h, int hidden, const __nv_bfloat16 *__restrict__ W_dkv,
+                      const __nv_bfloat16 *__restrict__ W_kr, const int *__restrict__ req,
+                      const int *__restrict__ pos, int n_tok, const int *__restrict__ page_table, int batch,
+                      int max_pages, int n_pages, float base, __nv_bfloat16 *__restrict__ cache, int *err) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    constexpr int D_C = 512, D_R = 64, D_ROW = 576;
+    extern __shared__ __align__(16) uint8_t asm_raw[];
+    const int ks = hidden / AP_SPLIT;                  // hidden slice of this CTA
+    const int ld = ks + 8;
+    __nv_bfloat16 *Ws = reinterpret_cast<__nv_bfloat16 *>(asm_raw);          // [64 cols][ks]
+    __nv_bfloat16 *Hs = Ws + AP_COLS * ld;                                    // [16 tok][ks]
+    float *part = reinterpret_cast<float *>(Hs + AP_TOK * ld);                // [16][64]
+    const int rank = (int)cluster.block_rank();
+    const int ct = blockIdx.x / AP_SPLIT, c0 = ct * AP_COLS, k0 = rank * ks;
+    const int t0 = blockIdx.y * AP_TOK;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    for (int c = tid; c < AP_COLS * ks / 8; c += 256) {
+        const int r = c / (ks / 8), k = (c % (ks / 8)) * 8, col = c0 + r;
+        const __nv_bfloat16 *src = col < D_C ? W_dkv + (size_t)col * hidden : W_kr + (size_t)(col - D_C) * hidden;
+        cp_async16(Ws + r * ld + k, src + k0 + k, true);
+    }
+    for (int c = tid; c < AP_TOK * ks / 8; c += 256) {
+        const int r = c / (ks / 8), k = (c % (ks / 8)) * 8, tok = t0 + r;
+        cp_async16(Hs + r * ld + k, h + (size_t)(tok < n_tok ? tok : 0) * hidden + k0 + k, tok < n_tok);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};   // warp w: tokens 0..15 x columns [8w, 8w + 8)
+    for (int kk = 0; kk < ks; kk += 32) {
+        uint32_t a0[4], a1[4], b[4];
+        ldmatrix_x4(a0[0], a0[1], a0[2], a0[3], Hs + ((lane % 8) + 8 * ((lane / 8) % 2)) * ld + kk + 8 * (lane / 16));
+        ldmatrix_x4(a1[0], a1[1], a1[2], a1[3],
+                    Hs + ((lane % 8) + 8 * ((lane / 8) % 2)) * ld + kk + 16 + 8 * (lane / 16));
+        ldmatrix_x4(b[0], b[1], b[2], b[3], Ws + (8 * warp + (lane % 8)) * ld + kk + 8 * (lane / 8));
+        mma_bf16(acc, a0, b[0], b[1]);
+        mma_bf16(acc, a1, b[2], b[3]);
+    }
+    const int gid = lane / 4, t4 = lane % 4;
+    part[gid * AP_COLS + 8 * warp + 2 * t4] = acc[0];
+    part[gid * AP_COLS + 8 * warp + 2 * t4 + 1] = acc[1];
+    part[(gid + 8) * AP_COLS + 8 * warp + 2 * t4] = acc[2];
+    part[(gid + 8) * AP_COLS + 8 * warp + 2 * t4 + 1] = acc[3];
+    cluster.sync();
+    if (rank == 0) {
+        for (int pi = tid; pi < AP_TOK * AP_COLS / 2; pi += 256) {
+            const int r = pi / (AP_COLS / 2), cp = pi % (AP_COLS / 2);
+            const int n = t0 + r, col = c0 + 2 * cp;
+            if (n >= n_tok) continue;
+            float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+            for (int q = 0; q < AP_SPLIT; ++q) {
+                const float *rp = cluster.map_shared_rank(part, q);
+                x0 += rp[r * AP_COLS + 2 * cp];
+                x1 += rp[r * AP_COLS + 2 * cp + 1];
+            }
+            const int b = req[n], p = pos[n];
+            if (b < 0 || b >= batch || p < 0 || p >= max_pages * 64) {
+                report(err, MLA_ERR_DEVICE_BOUNDS);
+                continue;
+            }
+            const int pid = page_table[(size_t)b * max_pages + p / 64];
+            if (pid < 0 || pid >= n_pages) {
+                report(err, MLA_ERR_DEVICE_BOUNDS);
+                continue;
+            }
+            if (col >= D_C) {
+                float cs, sn;
+                rope_cos_sin(p, (col - D_C) / 2, D_R, base, &cs, &sn);
+                const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
+                x0 = y0;
+                x1 = y1;
+            }
+            __nv_bfloat16 *dst = cache + ((size_t)pid * 64 + p % 64) * D_ROW + col;
+            *reinterpret_cast<uint32_t *>(dst) = pack_bf16(x0, x1);
+        }
+    }
+    cluster.sync();   // partner tiles stay alive until rank 0 has read them
+}
+
+}  // namespace
+
+bool append_mma_ok(const Dims &d, int hidden, bool projected) {
+    // hidden slices must be whole 32-column MMA steps, and the slice tiles must fit shared memory
+    return projected && d.bf16 && d.d_c == 512 && d.d_r == 64 && d.page == 64 && hidden % (32 * AP_SPLIT) == 0 &&
+           hidden >= 32 * AP_SPLIT && hidden <= 10240;
+}
+
+cudaError_t launch_append_mma(const Dims &d, const void *h, int hidden, const void *W_dkv, const void *W_kr,
+                              const int *req, const int *pos, int n_tok, const int *page_table, int batch,
+                              int max_pages, int n_pages, void *cache, int *err, cudaStream_t st) {
+    const int ks = hidden / AP_SPLIT, ld = ks + 8;
+    const size_t smem = sizeof(__nv_bfloat16) * (size_t)(AP_COLS + AP_TOK) * ld + sizeof(float) * AP_TOK * AP_COLS;
+    cudaError_t e = cudaFuncSetAttribute(append_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(9 * AP_SPLIT, ceil_div(n_tok, AP_TOK));
+    append_mma_kernel<<<grid, 256, smem, st>>>((const __nv_bfloat16 *)h, hidden, (const __nv_bfloat16 *)W_dkv,
+                                               (const __nv_bfloat16 *)W_kr, req, pos, n_tok, page_table, batch,
+                                               max_pages, n_pages, d.base, (__nv_bfloat16 *)cache, err);
+    return cudaGetLastError();
+}
+
+}  // namespace mla

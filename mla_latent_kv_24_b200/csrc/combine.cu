@@ -91,3 +91,148 @@ cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part
 }
 
 }  // namespace mla
+
+// ---------------------------------------------------------------------------------------
+// Tensor-core combine + W_UV for the DeepSeek-V2 shape (bf16, d_c = 512, d_v = 128).  One CTA
+// takes one head and 32 query rows: it merges each row's chunk partials into bf16 latent rows
+// in shared memory (the same exact merge as above), then computes out[rows, 128] =
+// O[rows, 512] W_UV[w]^T with mma.sync m16n8k16, streaming W_UV[w] in four 128-column slices
+// through a double-buffered cp.async ring.  W_UV is read once per head (16.8 MB for H = 128)
+// and the fp32 partials once.
+// ---------------------------------------------------------------------------------------
+#include "warp_mma.cuh"
+
+namespace mla {
+namespace {
+
+constexpr int CM = 32, CN = 128, CK = 512, CKC = 128, O_LD = CK + 8, W_LD = CKC + 8;
+
+__global__ void __launch_bounds__(256) combine_mma_kernel(const float *__restrict__ part_o,
+                                                          const float *__restrict__ part_ml,
+                                                          const int *__restrict__ row_first, int rows, int H,
+                                                          const __nv_bfloat16 *__restrict__ W_uv, int hpw,
+                                                          __nv_bfloat16 *__restrict__ out) {
+    extern __shared__ __align__(16) __nv_bfloat16 csm[];
+    __nv_bfloat16 *Os = csm;                       // [64][512 + 8]
+    __nv_bfloat16 *Ws = csm + CM * O_LD;           // [2][128 v][128 + 8]
+    const int h = blockIdx.x, row0 = blockIdx.y * CM;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const __nv_bfloat16 *W = W_uv + (size_t)(h / hpw) * CN * CK;
+    auto load_w = [&](int s, int c0) {
+        for (int c = tid; c < CN * CKC / 8; c += 256) {   // 2048 chunks of 16 B
+            const int v = c / (CKC / 8), k = (c % (CKC / 8)) * 8;
+            cp_async16(Ws + (s * CN + v) * W_LD + k, W + (size_t)v * CK + c0 + k, true);
+        }
+        cp_async_commit();
+    };
+    load_w(0, 0);
+    // Merge the chunk partials of every row of this tile: warp w takes rows w, w + 8, ...; lane
+    // l owns latent columns [16 l, 16 l + 16).
+    for (int r = warp; r < CM; r += 8) {
+        const int row = row0 + r;
+        float4 acc4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (row < rows) {
+            const int k0 = row_first[row], k1 = row_first[row + 1];
+            float M = -INFINITY;
+            for (int k = k0 + lane; k < k1; k += 32) M = fmaxf(M, part_ml[((size_t)k * H + h) * 2]);
+#pragma unroll
+            for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            float den = 0.f;
+#pragma unroll 2
+            for (int k = k0; k < k1; ++k) {
+                const float2 ml = *reinterpret_cast<const float2 *>(part_ml + ((size_t)k * H + h) * 2);
+                const float wk = ml.x == -INFINITY ? 0.f : expf(ml.x - M);
+                den += wk * ml.y;
+                const float4 *po = reinterpret_cast<const float4 *>(part_o + ((size_t)k * H + h) * CK + 16 * lane);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 v = po[q];
+                    acc4[q].x += wk * v.x;
+                    acc4[q].y += wk * v.y;
+                    acc4[q].z += wk * v.z;
+                    acc4[q].w += wk * v.w;
+                }
+            }
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc4[q].x *= inv;
+                acc4[q].y *= inv;
+                acc4[q].z *= inv;
+                acc4[q].w *= inv;
+            }
+        }
+        uint4 pk0 = make_uint4(pack_bf16(acc4[0].x, acc4[0].y), pack_bf16(acc4[0].z, acc4[0].w),
+                               pack_bf16(acc4[1].x, acc4[1].y), pack_bf16(acc4[1].z, acc4[1].w));
+        uint4 pk1 = make_uint4(pack_bf16(acc4[2].x, acc4[2].y), pack_bf16(acc4[2].z, acc4[2].w),
+                               pack_bf16(acc4[3].x, acc4[3].y), pack_bf16(acc4[3].z, acc4[3].w));
+        *reinterpret_cast<uint4 *>(Os + r * O_LD + 16 * lane) = pk0;
+        *reinterpret_cast<uint4 *>(Os + r * O_LD + 16 * lane + 8) = pk1;
+    }
+    const int wm = warp % 2, wn = warp / 2;   // warp tile 16 rows x 32 columns
+    float acc[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
+    for (int kc = 0; kc < CK / CKC; ++kc) {
+        if (kc + 1 < CK / CKC) {
+            load_w((kc + 1) & 1, (kc + 1) * CKC);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const __nv_bfloat16 *Wt = Ws + (kc & 1) * CN * W_LD;
+#pragma unroll
+        for (int kk = 0; kk < CKC; kk += 16) {
+            uint32_t a[4];
+            ldmatrix_x4(a[0], a[1], a[2], a[3],
+                        Os + (wm * 16 + (lane % 8) + 8 * ((lane / 8) % 2)) * O_LD + kc * CKC + kk + 8 * (lane / 16));
+#pragma unroll
+            for (int j = 0; j < 4; j += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldmatrix_x4(b0, b1, b2, b3,
+                            Wt + (wn * 32 + j * 8 + (lane % 8) + 8 * (lane / 16)) * W_LD + kk + 8 * ((lane / 8) % 2));
+                mma_bf16(acc[j], a, b0, b1);
+                mma_bf16(acc[j + 1], a, b2, b3);
+            }
+        }
+        __syncthreads();   // the next load overwrites this slice's buffer
+    }
+    const int gid = lane / 4, t4 = lane % 4;
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+        const int row = row0 + wm * 16 + gid + 8 * hr;
+        if (row >= rows) continue;
+        __nv_bfloat16 *dst = out + ((size_t)row * H + h) * CN + wn * 32;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint32_t *>(dst + j * 8 + 2 * t4) = pack_bf16(acc[j][2 * hr], acc[j][2 * hr + 1]);
+    }
+}
+
+}  // namespace
+
+bool combine_mma_ok(const Dims &d, int DV, bool project) {
+    return project && d.bf16 && DV == CK && d.d_v == CN;
+}
+
+cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
+                               int rows, const void *W_uv, void *out, cudaStream_t st) {
+    const size_t smem = sizeof(__nv_bfloat16) * ((size_t)CM * O_LD + 2 * (size_t)CN * W_LD);
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(combine_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    dim3 grid(d.H, ceil_div(rows, CM));
+    combine_mma_kernel<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, d.H, (const __nv_bfloat16 *)W_uv,
+                                                d.hpw, (__nv_bfloat16 *)out);
+    return cudaGetLastError();
+}
+
+}  // namespace mla

@@ -22,6 +22,12 @@ cudaError_t launch_append(const Dims &d, const void *h, int hidden, const void *
                           const int *page_table, int batch, int max_pages, int n_pages,
                           void *cache, int *err, cudaStream_t st);
 
+// Tensor-core append (bf16, d_c = 512, d_rope = 64, page 64, projected input) (append.cu).
+bool append_mma_ok(const Dims &d, int hidden, bool projected);
+cudaError_t launch_append_mma(const Dims &d, const void *h, int hidden, const void *W_dkv, const void *W_kr,
+                              const int *req, const int *pos, int n_tok, const int *page_table, int batch,
+                              int max_pages, int n_pages, void *cache, int *err, cudaStream_t st);
+
 // Split plan from device seq_lens (plan.cu).
 cudaError_t launch_plan(const int *seq_lens, int batch, int s_q, int max_pages, int page,
                         int chunk, int n_work_expected, WorkItem *items, int *row_first,
@@ -31,6 +37,11 @@ cudaError_t launch_plan(const int *seq_lens, int batch, int s_q, int max_pages, 
 //   q_abs [rows, H, d_c + d_r] = [W_UK[w]^T q_nope | RoPE(q_rope, p)], rows = batch * s_q.
 cudaError_t launch_q_absorb(const Dims &d, const void *q, const void *W_uk, const int *seq_lens,
                             int batch, int s_q, void *q_abs, cudaStream_t st);
+
+// Tensor-core variant for bf16, d_nope = 128, d_c = 512, d_rope = 64 (absorb.cu).
+bool q_absorb_mma_ok(const Dims &d);
+cudaError_t launch_q_absorb_mma(const Dims &d, const void *q, const void *W_uk, const int *seq_lens, int batch,
+                                int s_q, void *q_abs, cudaStream_t st);
 
 // RoPE of the query's RoPE part only (absorb.cu): q_rot [rows, H, d_n + d_r].
 cudaError_t launch_q_rope(const Dims &d, const void *q, const int *seq_lens, int batch, int s_q,
@@ -57,6 +68,11 @@ int simt_heads_per_block(const Dims &d, int mode);
 cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part_ml,
                            const int *row_first, int rows, int DV, const void *W_uv, void *out,
                            cudaStream_t st);
+
+// Tensor-core combine + W_UV for bf16, d_c = 512, d_v = 128 (combine.cu).
+bool combine_mma_ok(const Dims &d, int DV, bool project);
+cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
+                               int rows, const void *W_uv, void *out, cudaStream_t st);
 
 // Per-group cache expansion (expand.cu).
 cudaError_t launch_expand(const Dims &d, const void *W_uk, const void *W_uv, const void *latent,
