@@ -127,9 +127,12 @@ mla_status check_batch(const Dims &d, int batch, int s_q, int max_pages, const i
 }
 
 // Workspace layout of one decode call.
+// Plan rows are (request, query) pairs, except on the tensor-core grouped path, where one work
+// item covers all s_q queries of a request (they share every K/V tile), so the plan has one
+// row per request and each item stores s_q partial results (qpi = queries per item).
 struct Layout {
     size_t q_off, items_off, row_off, po_off, pml_off, total;
-    int n_work, chunk, rows, DK, DV;
+    int n_work, chunk, rows, plan_sq, qpi, DK, DV;
     bool tc;
 };
 
@@ -154,19 +157,21 @@ mla_status make_layout(const Dims &d, Path path, bool tc, int sms, int batch, in
         units = std::max(1, 4 * sms / std::max(1, d.H / hb));
         granule = 32;
     }
-    L->chunk = plan_chunk(lens, batch, s_q, units, granule);
-    L->n_work = (int)plan_count(lens, batch, s_q, L->chunk);
+    L->plan_sq = (path == GROUPED && grouped_tc_ok(d)) ? 1 : s_q;
+    L->qpi = s_q / L->plan_sq;
+    L->chunk = plan_chunk(lens, batch, L->plan_sq, units, granule);
+    L->n_work = (int)plan_count(lens, batch, L->plan_sq, L->chunk);
     size_t off = 0;
     L->q_off = off;
     off = align256(off + (size_t)L->rows * d.H * L->DK * elt(d));
     L->items_off = off;
     off = align256(off + (size_t)L->n_work * sizeof(WorkItem));
     L->row_off = off;
-    off = align256(off + (size_t)(L->rows + 1) * sizeof(int));
+    off = align256(off + (size_t)(batch * L->plan_sq + 1) * sizeof(int));
     L->po_off = off;
-    off = align256(off + (size_t)L->n_work * d.H * L->DV * sizeof(float));
+    off = align256(off + (size_t)L->n_work * L->qpi * d.H * L->DV * sizeof(float));
     L->pml_off = off;
-    off = align256(off + (size_t)L->n_work * d.H * 2 * sizeof(float));
+    off = align256(off + (size_t)L->n_work * L->qpi * d.H * 2 * sizeof(float));
     L->total = off;
     return MLA_OK;
 }
@@ -309,9 +314,9 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
     float *part_o = (float *)(w + L.po_off);
     float *part_ml = (float *)(w + L.pml_off);
     void *qp = w + L.q_off;
-    Plan plan{items, row_first, L.n_work, L.rows, L.chunk};
+    Plan plan{items, row_first, L.n_work, batch * L.plan_sq, L.chunk};
 
-    MLA_CUDA(launch_plan(seq_lens, batch, s_q, max_pages, d.page, L.chunk, L.n_work, items, row_first, err, st),
+    MLA_CUDA(launch_plan(seq_lens, batch, L.plan_sq, max_pages, d.page, L.chunk, L.n_work, items, row_first, err, st),
              "launch plan");
     if (path == ABSORBED) {
         if (q_absorb_mma_ok(d))
@@ -332,7 +337,7 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
             MLA_CUDA(launch_combine_mma(d, part_o, part_ml, row_first, L.rows, W_uv, out, st),
                      "launch combine + W_UV (tensor cores)");
         else
-            MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, L.DV, W_uv, out, st), "launch combine");
+            MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, 1, L.DV, W_uv, out, st), "launch combine");
     } else {
         if (grouped_tc_ok(d)) {
             ProfileScope prof(st);
@@ -345,7 +350,7 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
             SimtDecodeArgs a{qp, latent, expanded, page_table, plan, max_pages, n_pages, s_q, 1, part_o, part_ml, err};
             MLA_CUDA(launch_decode_simt(d, a, st), "launch grouped decode (CUDA cores)");
         }
-        MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, L.DV, nullptr, out, st), "launch combine");
+        MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, L.qpi, L.DV, nullptr, out, st), "launch combine");
     }
     return MLA_OK;
 }

@@ -21,28 +21,30 @@ constexpr int RB = 8;
 template <typename T>
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ part_o,
                                                       const float *__restrict__ part_ml,
-                                                      const int *__restrict__ row_first, int rows, int H,
-                                                      int DV, const T *__restrict__ W_uv, int hpw, int d_v,
-                                                      T *__restrict__ out) {
+                                                      const int *__restrict__ row_first, int rows, int qpi,
+                                                      int H, int DV, const T *__restrict__ W_uv, int hpw,
+                                                      int d_v, T *__restrict__ out) {
     extern __shared__ float O[];  // [RB][DV]
     const int h = blockIdx.x;
     const int row0 = blockIdx.y * RB;
     const int nr = min(RB, rows - row0);
     for (int r = 0; r < nr; ++r) {
-        const int k0 = row_first[row0 + r], k1 = row_first[row0 + r + 1];
+        const int pr = (row0 + r) / qpi, j = (row0 + r) % qpi;
+        const int k0 = row_first[pr], k1 = row_first[pr + 1];
+        auto ml = [&](int k, int e) { return part_ml[(((size_t)k * qpi + j) * H + h) * 2 + e]; };
         float M = -INFINITY;
-        for (int k = k0; k < k1; ++k) M = fmaxf(M, part_ml[((size_t)k * H + h) * 2]);
+        for (int k = k0; k < k1; ++k) M = fmaxf(M, ml(k, 0));
         float den = 0.f;
         for (int k = k0; k < k1; ++k) {
-            const float mk = part_ml[((size_t)k * H + h) * 2];
-            if (mk != -INFINITY) den += expf(mk - M) * part_ml[((size_t)k * H + h) * 2 + 1];
+            const float mk = ml(k, 0);
+            if (mk != -INFINITY) den += expf(mk - M) * ml(k, 1);
         }
         const float inv = den > 0.f ? 1.f / den : 0.f;
         for (int c = threadIdx.x; c < DV; c += blockDim.x) {
             float num = 0.f;
             for (int k = k0; k < k1; ++k) {
-                const float mk = part_ml[((size_t)k * H + h) * 2];
-                if (mk != -INFINITY) num += expf(mk - M) * part_o[((size_t)k * H + h) * DV + c];
+                const float mk = ml(k, 0);
+                if (mk != -INFINITY) num += expf(mk - M) * part_o[(((size_t)k * qpi + j) * H + h) * DV + c];
             }
             O[r * DV + c] = num * inv;
         }
@@ -73,18 +75,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 }  // namespace
 
 cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
-                           int rows, int DV, const void *W_uv, void *out, cudaStream_t st) {
+                           int rows, int qpi, int DV, const void *W_uv, void *out, cudaStream_t st) {
     dim3 grid(d.H, ceil_div(rows, RB));
     const size_t smem = sizeof(float) * RB * DV;
     if (d.bf16) {
         auto k = combine_kernel<__nv_bfloat16>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, d.H, DV, (const __nv_bfloat16 *)W_uv,
+        k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV, (const __nv_bfloat16 *)W_uv,
                                    d.hpw, d.d_v, (__nv_bfloat16 *)out);
     } else {
         auto k = combine_kernel<float>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, d.H, DV, (const float *)W_uv, d.hpw, d.d_v,
+        k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV, (const float *)W_uv, d.hpw, d.d_v,
                                    (float *)out);
     }
     return cudaGetLastError();

@@ -1,14 +1,304 @@
-// Grouped (GQA-path) tensor-core decode (not built yet: the CUDA-core kernel runs meanwhile).
+// GQA-path split decode over the per-group expanded cache ("GQLA: Group-Query Latent Attention
+// ..." abstract: the GQA path with a per-group expanded cache; AI Radio episode transcript:
+// per-group K and V plus the shared RoPE key).  For query j of request b (position p_j) and
+// head h of group g = h / 8:
+//     s_t = scale * ([q_nope | RoPE(q_rope, p_j)] . [K_g,t | k^R_t]),  t <= p_j
+//     o   = sum_t softmax(s)_t V_g,t
+//
+// The path is bound by HBM (8320 bytes per token for 16 groups, ~10 flop per byte per query),
+// so the kernel streams the expanded cache with deep cp.async pipelines and uses warp-level
+// mma.sync (m16n8k16, fp32 accumulators), whose throughput is far above what the bytes need.
+// One CTA takes one chunk of one request and one group: the group's 8 heads of every query of
+// the request form the 16 rows of the MMA tile (both MTP queries share each K/V tile), so each
+// page of K_g|V_g (32 KiB, contiguous) and of k^R (8 KiB) is read once per chunk.  Four warps
+// each take 16 tokens of every 64-token page and keep their own online softmax; the CTA merges
+// the four (m, l, O) at the end and writes one partial result per query for the combine.
+#include <math.h>
+
 #include "tc_decode.h"
+#include "warp_mma.cuh"
 
 namespace mla {
+namespace {
 
-bool grouped_tc_ok(const Dims &) { return false; }
-int grouped_units(const Dims &, int sms) { return sms; }
-int grouped_token_granule() { return 64; }
-cudaError_t launch_grouped_decode(const Dims &, const void *, const void *, const void *, const int *, const int *,
-                                  const Plan &, int, int, int, float *, float *, int *, cudaStream_t) {
-    return cudaErrorNotSupported;
+constexpr int GH = 8;                 // heads per group
+constexpr int D_N = 128, D_V = 128, D_R = 64, D_QK = 192, D_LAT = 512, D_ROW = 576, PAGE = 64;
+constexpr int KV_LD = 256 + 8;        // padded [K | V] row (elements)
+constexpr int KR_LD = 64 + 8;         // padded k^R row
+constexpr int Q_LD = D_QK + 8;        // padded query row
+constexpr int STAGES = 2;
+constexpr int WARPS = 4;
+constexpr int KV_TILE = PAGE * KV_LD, KR_TILE = PAGE * KR_LD;
+// The final cross-warp reduction reuses the stage buffers (all copies have landed by then).
+constexpr size_t STAGE_BYTES = sizeof(__nv_bfloat16) * STAGES * (KV_TILE + KR_TILE);
+constexpr size_t RED_BYTES = sizeof(float) * WARPS * 16 * (2 + D_V);
+static_assert(RED_BYTES <= STAGE_BYTES, "reduction buffer must fit in the stage buffers");
+constexpr size_t SMEM = STAGE_BYTES + sizeof(__nv_bfloat16) * 16 * Q_LD;   // 92416 B: 2 CTAs per SM
+
+struct GParams {
+    const __nv_bfloat16 *q, *expanded, *latent;
+    const int *page_table, *seq_lens;
+    Plan plan;
+    int max_pages, n_pages, s_q, H;
+    float scale_log2, base;
+    float *part_o, *part_ml;   // [n_work * s_q, H, 128], [n_work * s_q, H, 2]
+    int *err;
+};
+
+__global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p) {
+    extern __shared__ __align__(16) uint8_t gsm[];
+    __nv_bfloat16 *kv = reinterpret_cast<__nv_bfloat16 *>(gsm);           // [STAGES][64][KV_LD]
+    __nv_bfloat16 *kr = kv + STAGES * KV_TILE;                            // [STAGES][64][KR_LD]
+    __nv_bfloat16 *qs = kr + STAGES * KR_TILE;                            // [16][Q_LD]
+    float *red_ml = reinterpret_cast<float *>(gsm);                       // [WARPS][16][2], after the loop
+    float *red_o = red_ml + WARPS * 16 * 2;                               // [WARPS][16][128], after the loop
+
+    const WorkItem it = p.plan.items[blockIdx.x];
+    const int g = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int b = it.row;                   // the plan of this path has one row per request
+    const int L = p.seq_lens[b];
+    const int G = p.H / GH;
+    const int n_pg = ceil_div(it.t1 - it.t0, PAGE);
+    const size_t part_base = (size_t)blockIdx.x * p.s_q;
+
+    if (it.t1 <= it.t0) {   // only in a rejected plan
+        for (int i = tid; i < p.s_q * GH; i += blockDim.x) {
+            const size_t r = part_base + i / GH;
+            p.part_ml[(r * p.H + g * GH + i % GH) * 2] = -INFINITY;
+            p.part_ml[(r * p.H + g * GH + i % GH) * 2 + 1] = 0.f;
+        }
+        return;
+    }
+    // Queries of this group: row m = j * 8 + hh (s_q = 2 fills all 16 rows, s_q = 1 the first 8).
+    for (int i = tid; i < 16 * (D_QK / 2); i += blockDim.x) {
+        const int m = i / (D_QK / 2), c = 2 * (i % (D_QK / 2));
+        const int j = m / GH, h = g * GH + m % GH;
+        float x0 = 0.f, x1 = 0.f;
+        if (j < p.s_q) {
+            const __nv_bfloat16 *src = p.q + (((size_t)b * p.s_q + j) * p.H + h) * D_QK + c;
+            x0 = __bfloat162float(src[0]);
+            x1 = __bfloat162float(src[1]);
+            if (c >= D_N) {
+                float cs, sn;
+                rope_cos_sin(L - p.s_q + j, (c - D_N) / 2, D_R, p.base, &cs, &sn);
+                const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
+                x0 = y0;
+                x1 = y1;
+            }
+        }
+        *reinterpret_cast<uint32_t *>(qs + m * Q_LD + c) = pack_bf16(x0, x1);
+    }
+    __syncthreads();
+
+    // Page i of the chunk into stage `stage`.  Rows past the chunk's end (the ragged last page)
+    // and the rows of an out-of-range page id are zero-filled, so stale slot contents (even
+    // non-finite ones) never reach P.V, where a zero probability would not cancel them.
+    auto load_page = [&](int stage, int i) {
+        int pid = p.page_table[(size_t)b * p.max_pages + it.t0 / PAGE + i];
+        bool ok = true;
+        if (pid < 0 || pid >= p.n_pages) {
+            if (tid == 0) report(p.err, MLA_ERR_DEVICE_BOUNDS);
+            ok = false;
+            pid = 0;
+        }
+        const int valid = ok ? min(PAGE, it.t1 - (it.t0 + PAGE * i)) : 0;
+        const __nv_bfloat16 *src_kv = p.expanded + (((size_t)pid * G + g) * PAGE) * 256;
+        const __nv_bfloat16 *src_kr = p.latent + ((size_t)pid * PAGE) * D_ROW + D_LAT;
+        __nv_bfloat16 *dkv = kv + stage * KV_TILE, *dkr = kr + stage * KR_TILE;
+        for (int c = tid; c < PAGE * 32; c += blockDim.x) {       // 64 rows x 32 chunks of 16 B
+            const int r = c / 32, k = (c % 32) * 8;
+            cp_async16(dkv + r * KV_LD + k, src_kv + (size_t)r * 256 + k, r < valid);
+        }
+        for (int c = tid; c < PAGE * 8; c += blockDim.x) {        // 64 rows x 8 chunks
+            const int r = c / 8, k = (c % 8) * 8;
+            cp_async16(dkr + r * KR_LD + k, src_kr + (size_t)r * D_ROW + k, r < valid);
+        }
+    };
+
+    // Query A fragments stay in registers for the whole chunk (12 k-steps of 16 dims).
+    uint32_t qa[12][4];
+#pragma unroll
+    for (int ks = 0; ks < 12; ++ks)
+        ldmatrix_x4(qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3],
+                    qs + ((lane % 8) + 8 * ((lane / 8) % 2)) * Q_LD + 16 * ks + 8 * (lane / 16));
+
+    const int gid = lane / 4, t4 = lane % 4;
+    // Rows gid and gid + 8 of this thread's fragments: query index and visible length.
+    const int lim0 = (gid / GH < p.s_q) ? L - p.s_q + gid / GH : -1;            // rows 0..7: query 0
+    const int lim1 = ((gid + 8) / GH < p.s_q) ? L - p.s_q + (gid + 8) / GH : -1; // rows 8..15: query 1
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float o[16][4];
+#pragma unroll
+    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+
+    load_page(0, 0);
+    cp_async_commit();
+    for (int i = 0; i < n_pg; ++i) {
+        if (i + 1 < n_pg) load_page((i + 1) % STAGES, i + 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        const __nv_bfloat16 *tkv = kv + (i % STAGES) * KV_TILE + (16 * warp) * KV_LD;
+        const __nv_bfloat16 *tkr = kr + (i % STAGES) * KR_TILE + (16 * warp) * KR_LD;
+        // S [16 rows x 16 tokens] = Q~ K~^T over 192 dims.
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < 12; ks += 2) {
+            // B fragments: rows = tokens, dims contiguous; x4 covers 2 k-steps of one n8 tile.
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                uint32_t bf[4];
+                const int tok = 8 * nt + (lane % 8);
+                const __nv_bfloat16 *src = ks < 8 ? tkv + tok * KV_LD + 16 * ks + 8 * (lane / 8)
+                                                  : tkr + tok * KR_LD + 16 * (ks - 8) + 8 * (lane / 8);
+                ldmatrix_x4(bf[0], bf[1], bf[2], bf[3], src);
+                mma_bf16(s[nt], qa[ks], bf[0], bf[1]);
+                mma_bf16(s[nt], qa[ks + 1], bf[2], bf[3]);
+            }
+        }
+        // Mask, scale, online softmax per row (rows gid and gid + 8; 4 tokens per row here).
+        const int tok_base = it.t0 + PAGE * i + 16 * warp;
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int t = tok_base + 8 * nt + 2 * t4 + e;
+                const bool in = t < it.t1;
+                s[nt][e] = (in && t <= lim0) ? s[nt][e] * p.scale_log2 : -INFINITY;
+                s[nt][2 + e] = (in && t <= lim1) ? s[nt][2 + e] * p.scale_log2 : -INFINITY;
+                mx0 = fmaxf(mx0, s[nt][e]);
+                mx1 = fmaxf(mx1, s[nt][2 + e]);
+            }
+#pragma unroll
+        for (int off = 1; off <= 2; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        const float a0 = n0 == -INFINITY ? 1.f : exp2f(m0 - n0), a1 = n1 == -INFINITY ? 1.f : exp2f(m1 - n1);
+        float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                s[nt][e] = n0 == -INFINITY ? 0.f : exp2f(s[nt][e] - n0);
+                s[nt][2 + e] = n1 == -INFINITY ? 0.f : exp2f(s[nt][2 + e] - n1);
+                sum0 += s[nt][e];
+                sum1 += s[nt][2 + e];
+            }
+        l0 = l0 * a0 + sum0;
+        l1 = l1 * a1 + sum1;
+        m0 = n0;
+        m1 = n1;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            o[n][0] *= a0;
+            o[n][1] *= a0;
+            o[n][2] *= a1;
+            o[n][3] *= a1;
+        }
+        // P (accumulator layout of S) is the A fragment of P.V (rows x 16 tokens).
+        uint32_t pa[4] = {pack_bf16(s[0][0], s[0][1]), pack_bf16(s[0][2], s[0][3]), pack_bf16(s[1][0], s[1][1]),
+                          pack_bf16(s[1][2], s[1][3])};
+        // O [16 x 128] += P V: V rows = tokens with v contiguous; .trans gives B fragments.
+#pragma unroll
+        for (int n = 0; n < 16; n += 2) {
+            uint32_t vb[4];
+            const __nv_bfloat16 *src = tkv + ((lane % 8) + 8 * ((lane / 8) % 2)) * KV_LD + D_N + 8 * n + 8 * (lane / 16);
+            ldmatrix_x4_trans(vb[0], vb[1], vb[2], vb[3], src);
+            mma_bf16(o[n], pa, vb[0], vb[1]);
+            mma_bf16(o[n + 1], pa, vb[2], vb[3]);
+        }
+        __syncthreads();   // this stage is refilled by the next iteration's load
+    }
+    cp_async_wait<0>();
+    __syncthreads();   // the stage buffers become the reduction buffer
+
+    // Merge the four warps' partial softmaxes: row sums over the 4 threads of each row first.
+#pragma unroll
+    for (int off = 1; off <= 2; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+    }
+    if (t4 == 0) {
+        red_ml[(warp * 16 + gid) * 2] = m0;
+        red_ml[(warp * 16 + gid) * 2 + 1] = l0;
+        red_ml[(warp * 16 + gid + 8) * 2] = m1;
+        red_ml[(warp * 16 + gid + 8) * 2 + 1] = l1;
+    }
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        red_o[(warp * 16 + gid) * D_V + 8 * n + 2 * t4] = o[n][0];
+        red_o[(warp * 16 + gid) * D_V + 8 * n + 2 * t4 + 1] = o[n][1];
+        red_o[(warp * 16 + gid + 8) * D_V + 8 * n + 2 * t4] = o[n][2];
+        red_o[(warp * 16 + gid + 8) * D_V + 8 * n + 2 * t4 + 1] = o[n][3];
+    }
+    __syncthreads();
+    // 16 rows x 128 columns; rows past s_q * 8 are padding.
+    for (int i = tid; i < 16 * D_V; i += blockDim.x) {
+        const int m = i / D_V, c = i % D_V, j = m / GH;
+        if (j >= p.s_q) continue;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) M = fmaxf(M, red_ml[(w * 16 + m) * 2]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) {
+            const float mw = red_ml[(w * 16 + m) * 2];
+            const float wt = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            num += wt * red_o[(w * 16 + m) * D_V + c];
+            den += wt * red_ml[(w * 16 + m) * 2 + 1];
+        }
+        const size_t r = part_base + j;
+        const int h = g * GH + m % GH;
+        p.part_o[(r * p.H + h) * D_V + c] = num;   // relative to max M (log2 units)
+        if (c == 0) {
+            p.part_ml[(r * p.H + h) * 2] = M * 0.69314718055994531f;
+            p.part_ml[(r * p.H + h) * 2 + 1] = den;
+        }
+    }
+}
+
+}  // namespace
+
+bool grouped_tc_ok(const Dims &d) {
+    return d.bf16 && d.hpw == GH && d.d_n == D_N && d.d_v == D_V && d.d_r == D_R && d.d_c == D_LAT && d.page == PAGE &&
+           d.H % GH == 0;
+}
+int grouped_units(const Dims &d, int sms) { return std::max(1, 8 * 2 * sms / std::max(1, d.H / GH)); }
+int grouped_token_granule() { return PAGE; }
+
+cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expanded, const void *latent,
+                                  const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
+                                  int n_pages, int s_q, float *part_o, float *part_ml, int *err, cudaStream_t st) {
+    if (plan.n_work == 0) return cudaSuccess;
+    GParams p;
+    p.q = (const __nv_bfloat16 *)q;
+    p.expanded = (const __nv_bfloat16 *)expanded;
+    p.latent = (const __nv_bfloat16 *)latent;
+    p.page_table = page_table;
+    p.seq_lens = seq_lens;
+    p.plan = plan;
+    p.max_pages = max_pages;
+    p.n_pages = n_pages;
+    p.s_q = s_q;
+    p.H = d.H;
+    p.scale_log2 = d.scale * 1.4426950408889634f;
+    p.base = d.base;
+    p.part_o = part_o;
+    p.part_ml = part_ml;
+    p.err = err;
+    static bool attr = false;
+    if (!attr) {
+        cudaError_t e = cudaFuncSetAttribute(grouped_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+        if (e != cudaSuccess) return e;
+        attr = true;
+    }
+    dim3 grid(plan.n_work, d.H / GH);
+    grouped_decode_kernel<<<grid, WARPS * 32, SMEM, st>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace mla

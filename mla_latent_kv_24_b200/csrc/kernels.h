@@ -64,9 +64,10 @@ cudaError_t launch_decode_simt(const Dims &d, const SimtDecodeArgs &a, cudaStrea
 int simt_heads_per_block(const Dims &d, int mode);
 
 // Split combine (+ W_UV up-projection when W_uv != nullptr) (combine.cu).
-//   out [rows, H, d_v]
+//   out [rows, H, d_v].  Output row r = (b, j) merges plan row r / qpi: partial results
+//   k * qpi + r % qpi for its work items k (qpi = 1 when every plan row is one query).
 cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part_ml,
-                           const int *row_first, int rows, int DV, const void *W_uv, void *out,
+                           const int *row_first, int rows, int qpi, int DV, const void *W_uv, void *out,
                            cudaStream_t st);
 
 // Tensor-core combine + W_UV for bf16, d_c = 512, d_v = 128 (combine.cu).

@@ -79,6 +79,32 @@ def test_grouped_small_shapes_match_oracle(B, s_q, lens):
     assert_close(wl.from_torch_f64(dev.decode_absorbed()), ref, "bf16", "absorbed on GQLA weights")
 
 
+@pytest.mark.parametrize("B,s_q,lens", [(1, 2, (5000,)), (4, 2, (129, 4097, 64, 3000)), (6, 1, (1, 63, 64, 65, 700, 2049))])
+def test_grouped_multi_chunk_shapes_match_oracle(B, s_q, lens):
+    # few requests against a whole GPU: every request is cut into many chunks, some of which end
+    # between the two queries' visible lengths
+    w = wl.small_workload(wl.WORKLOADS["5_8192_1"], B=B, s_q=s_q, lens=list(lens), shuffle_pages=True, seed=131 + B)
+    inp = wl.make_inputs(w)
+    dev = Dev(inp)
+    got = wl.from_torch_f64(dev.decode_grouped(dev.expand()))
+    assert_close(got, oracle_decode(inp), "bf16", f"grouped multi-chunk {lens}")
+
+
+def test_grouped_ignores_nonfinite_stale_slots():
+    # slots past a request's length in its last page are never read as keys or values
+    w = wl.small_workload(wl.WORKLOADS["5_8192_1"], B=3, s_q=2, lens=[70, 130, 1000], shuffle_pages=True, seed=21)
+    inp = wl.make_inputs(w)
+    dev = Dev(inp)
+    exp = dev.expand()
+    for b, L in enumerate(inp.seq_lens):
+        last = int(inp.page_table[b, (int(L) - 1) // w.page])
+        used = int(L) - ((int(L) - 1) // w.page) * w.page
+        exp[last, :, used:, :] = float("nan")
+        dev.cache.view(inp.n_pages, w.page, w.d_row)[last, used:, :] = float("nan")
+    got = wl.from_torch_f64(dev.decode_grouped(exp))
+    assert_close(got, oracle_decode(inp), "bf16", "grouped with NaN stale slots")
+
+
 def test_expand_cache_matches_oracle():
     import oracle
     w = wl.small_workload(wl.WORKLOADS["5_8192_1"], B=2, lens=[100, 64], seed=5)
