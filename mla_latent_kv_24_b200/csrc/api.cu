@@ -334,10 +334,12 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
             MLA_CUDA(launch_decode_simt(d, a, st), "launch decode (CUDA cores)");
         }
         if (combine_mma_ok(d, L.DV, true))
-            MLA_CUDA(launch_combine_mma(d, part_o, part_ml, row_first, L.rows, W_uv, out, st),
+            MLA_CUDA(launch_combine_mma(d, part_o, part_ml, row_first, L.rows, tc, W_uv, out, st),
                      "launch combine + W_UV (tensor cores)");
-        else
+        else if (!tc)
             MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, 1, L.DV, W_uv, out, st), "launch combine");
+        else
+            return fail(MLA_ERR_UNSUPPORTED, "tcgen05 partials need the tensor-core combine");
     } else {
         if (grouped_tc_ok(d)) {
             ProfileScope prof(st);

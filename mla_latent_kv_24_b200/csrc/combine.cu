@@ -109,6 +109,8 @@ namespace {
 
 constexpr int CM = 32, CN = 128, CK = 512, CKC = 128, O_LD = CK + 8, W_LD = CKC + 8;
 
+// OCT: partials in the column-octet layout [k][64][H][8] of the tcgen05 decode (else [k][H][512]).
+template <bool OCT>
 __global__ void __launch_bounds__(256) combine_mma_kernel(const float *__restrict__ part_o,
                                                           const float *__restrict__ part_ml,
                                                           const int *__restrict__ row_first, int rows, int H,
@@ -148,9 +150,11 @@ __global__ void __launch_bounds__(256) combine_mma_kernel(const float *__restric
                 const float wk = ml.x == -INFINITY ? 0.f : expf(ml.x - M);
                 den += wk * ml.y;
                 const float4 *po = reinterpret_cast<const float4 *>(part_o + ((size_t)k * H + h) * CK + 16 * lane);
+                const float4 *po0 = reinterpret_cast<const float4 *>(part_o + (((size_t)k * 64 + 2 * lane) * H + h) * 8);
+                const float4 *po1 = reinterpret_cast<const float4 *>(part_o + (((size_t)k * 64 + 2 * lane + 1) * H + h) * 8);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float4 v = po[q];
+                    const float4 v = OCT ? (q < 2 ? po0[q] : po1[q - 2]) : po[q];
                     acc4[q].x += wk * v.x;
                     acc4[q].y += wk * v.y;
                     acc4[q].z += wk * v.z;
@@ -223,17 +227,20 @@ bool combine_mma_ok(const Dims &d, int DV, bool project) {
 }
 
 cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
-                               int rows, const void *W_uv, void *out, cudaStream_t st) {
+                               int rows, bool oct_layout, const void *W_uv, void *out, cudaStream_t st) {
     const size_t smem = sizeof(__nv_bfloat16) * ((size_t)CM * O_LD + 2 * (size_t)CN * W_LD);
     static bool attr = false;
     if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(combine_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(combine_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(combine_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         attr = true;
     }
     dim3 grid(d.H, ceil_div(rows, CM));
-    combine_mma_kernel<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, d.H, (const __nv_bfloat16 *)W_uv,
-                                                d.hpw, (__nv_bfloat16 *)out);
+    auto k = oct_layout ? combine_mma_kernel<true> : combine_mma_kernel<false>;
+    k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, d.H, (const __nv_bfloat16 *)W_uv, d.hpw,
+                               (__nv_bfloat16 *)out);
     return cudaGetLastError();
 }
 

@@ -99,7 +99,7 @@ struct TcParams {
     const int *page_table;
     int max_pages, n_pages, s_q;
     float scale_log2;  // softmax scale * log2(e)
-    float *part_o;     // [n_work, H, 512]
+    float *part_o;     // [n_work, 64, H, 8]: column octet-major (see the epilogue)
     float *part_ml;    // [n_work, H, 2]: max (natural-log units), sum
     int *err;
 };
@@ -208,6 +208,8 @@ __device__ void run_v_producer(const Ctx &c, const TcParams &p, const CUtensorMa
 // report exactly its own work.
 __device__ void run_qk_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, int pair, int n_pairs) {
     int g = 0, item_n = 0;
+    const uint64_t qdesc = tc::sdesc_sw128(c.base + OFF_Q, 16, 1024);
+    const uint64_t kdesc = tc::sdesc_sw128(c.base + OFF_K, 16, 1024);
     for (int k = pair; k < p.plan.n_work; k += n_pairs) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) continue;   // only in a rejected plan, and then for every item
@@ -219,18 +221,22 @@ __device__ void run_qk_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
             if (g >= 2 && !wait_or_abort(c, c.bar(B_SFREE + sb), (uint32_t)((g - 2) >> 1) & 1u, p.err)) return;
             tc::fence_after_sync();
             const uint32_t d = tmem + TM_S + 64 * sb;
+#pragma unroll
             for (int j = 0; j < NK; ++j) {
                 if (!wait_or_abort(c, c.bar(B_KFULL + j), (uint32_t)g & 1u, p.err)) return;
                 tc::fence_after_sync();
-                for (int q3 = 0; q3 < 3; ++q3) {
-                    const int cb = 3 * j + q3;
+#pragma unroll
+                for (int q3 = 0; q3 < 3; ++q3)
 #pragma unroll
                     for (int w4 = 0; w4 < 4; ++w4) {
-                        const uint64_t a = tc::sdesc_sw128(c.base + OFF_Q + cb * BOX + 32 * w4, 16, 1024);
-                        const uint64_t bd = tc::sdesc_sw128(c.kslot(j) + q3 * BOX + 32 * w4, 16, 1024);
-                        tc::mma_pair_bf16(d, a, bd, IDESC_QK, (cb | w4) ? 1u : 0u);
+                        const int cb = 3 * j + q3;
+                        const uint64_t a = tc::sdesc_add(qdesc, cb * BOX + 32 * w4);
+                        const uint64_t bd = tc::sdesc_add(kdesc, j * KSLOT + q3 * BOX + 32 * w4);
+                        if (cb == 0 && w4 == 0)
+                            tc::mma_pair_bf16_k<false>(d, a, bd, IDESC_QK);
+                        else
+                            tc::mma_pair_bf16_k<true>(d, a, bd, IDESC_QK);
                     }
-                }
                 tc::commit_pair(c.bar(B_KEMPTY + j), 0x3);
             }
             if (i == n_steps - 1) tc::commit_pair(c.bar(B_QEMPTY), 0x3);
@@ -242,7 +248,9 @@ __device__ void run_qk_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
 
 __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, int pair, int n_pairs) {
     int g = 0, item_n = 0;
-    const uint32_t pbase = c.base + OFF_P;
+    const uint64_t pdesc = tc::sdesc_sw128(c.base + OFF_P, 16, 1024);
+    const uint64_t vdesc = tc::sdesc_sw128(c.base + OFF_V, BOX, 1024);
+    const uint32_t o_tmem = tmem + TM_O;
     for (int k = pair; k < p.plan.n_work; k += n_pairs) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) continue;
@@ -252,17 +260,21 @@ __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
             // The first PV of an item overwrites O: the previous item's epilogue must be done with it.
             if (i == 0 && item_n > 0 && !wait_or_abort(c, c.bar(B_OFREE), (uint32_t)(item_n - 1) & 1u, p.err)) return;
             tc::fence_after_sync();
+#pragma unroll
             for (int pg = 0; pg < NV; ++pg) {
                 if (!wait_or_abort(c, c.bar(B_VFULL + pg), (uint32_t)g & 1u, p.err)) return;
                 tc::fence_after_sync();
-                for (int ch = 0; ch < 2; ++ch) {
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint64_t a = tc::sdesc_sw128(pbase + pg * BOX + 32 * k4, 16, 1024);
-                        const uint64_t bd = tc::sdesc_sw128(c.vslot(pg) + 2 * BOX * ch + 2048 * k4, BOX, 1024);
-                        tc::mma_pair_bf16(tmem + TM_O + 128 * ch, a, bd, IDESC_PV, (i == 0 && pg == 0 && k4 == 0) ? 0u : 1u);
+                        const uint64_t a = tc::sdesc_add(pdesc, pg * BOX + 32 * k4);
+                        const uint64_t bd = tc::sdesc_add(vdesc, pg * VSLOT + 2 * BOX * ch + 2048 * k4);
+                        if (pg == 0 && k4 == 0 && i == 0)
+                            tc::mma_pair_bf16_k<false>(o_tmem + 128 * ch, a, bd, IDESC_PV);
+                        else
+                            tc::mma_pair_bf16_k<true>(o_tmem + 128 * ch, a, bd, IDESC_PV);
                     }
-                }
                 tc::commit_pair(c.bar(B_VEMPTY + pg), 0x3);
             }
             tc::commit_pair(c.bar(B_PVDONE + (g & 1)), 0x3);
@@ -383,15 +395,20 @@ __device__ void run_softmax(const Ctx &c, const TcParams &p, uint32_t tmem, int 
         float l1, l2, l3;
         others(g & 1, l_run, l1, l2, l3);
         const float l_tot = (l_run + l1) + (l2 + l3);
-        float *dst = p.part_o + ((size_t)k * H + head) * 512 + 256 * half + 128 * hsel;
+        // Partial O in the octet layout [item][64 column octets][H][8]: a warp (32 consecutive heads)
+        // stores 32 whole 32-byte sectors per octet, 1 KiB contiguous.
 #pragma unroll 1
         for (int q = 0; q < 2; ++q) {
             float v[64];
             tc::tmem_ld64(tmem + TM_O + 128 * half + 64 * q + lane_addr, v);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-                *reinterpret_cast<float4 *>(dst + 64 * q + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            for (int jo = 0; jo < 8; ++jo) {
+                const int oct = 32 * half + 16 * hsel + 8 * q + jo;
+                float4 *dst = reinterpret_cast<float4 *>(p.part_o + (((size_t)k * 64 + oct) * H + head) * 8);
+                dst[0] = make_float4(v[8 * jo], v[8 * jo + 1], v[8 * jo + 2], v[8 * jo + 3]);
+                dst[1] = make_float4(v[8 * jo + 4], v[8 * jo + 5], v[8 * jo + 6], v[8 * jo + 7]);
+            }
         }
         tc::fence_before_sync();
         __syncwarp();

@@ -70,10 +70,12 @@ cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part
                            const int *row_first, int rows, int qpi, int DV, const void *W_uv, void *out,
                            cudaStream_t st);
 
-// Tensor-core combine + W_UV for bf16, d_c = 512, d_v = 128 (combine.cu).
+// Tensor-core combine + W_UV for bf16, d_c = 512, d_v = 128 (combine.cu).  oct_layout: the
+// partials are in the tcgen05 decode's column-octet layout [n_work, 64, H, 8] instead of
+// [n_work, H, 512].
 bool combine_mma_ok(const Dims &d, int DV, bool project);
 cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
-                               int rows, const void *W_uv, void *out, cudaStream_t st);
+                               int rows, bool oct_layout, const void *W_uv, void *out, cudaStream_t st);
 
 // Per-group cache expansion (expand.cu).
 cudaError_t launch_expand(const Dims &d, const void *W_uk, const void *W_uv, const void *latent,

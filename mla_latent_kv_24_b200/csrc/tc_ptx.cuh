@@ -146,6 +146,18 @@ __device__ __forceinline__ void mma_pair_bf16(uint32_t d_tmem, uint64_t a_desc, 
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// Same with the accumulate flag fixed at compile time (no predicate set-up in the issue loop).
+template <bool ACCUMULATE>
+__device__ __forceinline__ void mma_pair_bf16_k(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
+    if (ACCUMULATE)
+        asm volatile("tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, 1;" ::"r"(d_tmem), "l"(a_desc), "l"(b_desc),
+                     "r"(idesc)
+                     : "memory");
+    else
+        asm volatile("tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, 0;" ::"r"(d_tmem), "l"(a_desc), "l"(b_desc),
+                     "r"(idesc)
+                     : "memory");
+}
 // Arrive (once) on the barrier at this shared-memory offset in every CTA of `cta_mask` when
 // all previously issued MMAs of this thread complete.
 __device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t cta_mask) {
@@ -236,6 +248,10 @@ __device__ __forceinline__ float ex2(float x) {
 // offsets (16-byte units), version 1, 128-byte swizzle.  K-major 128B-swizzled operands use
 // SBO = 1024 (eight 128-byte rows) and ignore LBO; MN-major ones use LBO = distance between
 // 64-element column blocks and SBO = 1024.
+// A descriptor's start address sits in its low 14 bits (in 16-byte units); shared memory is
+// below 256 KiB, so adding a byte offset / 16 to a descriptor moves its start address without
+// touching the other fields.  Issue loops build one descriptor per buffer and add constants.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t byte_offset) { return desc + (byte_offset >> 4); }
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
     uint64_t d = 0;
     d |= (uint64_t)((addr >> 4) & 0x3FFF);
