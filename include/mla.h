@@ -136,7 +136,10 @@ MLA_API mla_status mla_decode_workspace_size(const mla_dims *dims, int32_t batch
  *   q             device [batch, s_q, H, d_nope + d_rope]; RoPE part NOT yet rotated.
  *   W_uk          device [H / heads_per_group, d_nope, d_c].
  *   W_uv          device [H / heads_per_group, d_v, d_c].
- *   latent_cache  device [n_pages_total, page_size, d_c + d_rope].
+ *   latent_cache  device [n_pages_total, page_size, d_c + d_rope].  Slots past a request's
+ *                 length in its last page must hold finite values (any finite values, e.g. a
+ *                 zero-initialised pool): the tensor-core kernel multiplies their zero softmax
+ *                 weights with them, and 0 * NaN would reach the output.
  *   page_table    device [batch, max_pages];  seq_lens device [batch];
  *   seq_lens_host host   [batch], equal to the device copy; s_q <= seq_lens[b] <= max_pages*page.
  *   out           device [batch, s_q, H, d_v].

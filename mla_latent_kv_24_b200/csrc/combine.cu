@@ -144,22 +144,45 @@ __global__ void __launch_bounds__(256) combine_mma_kernel(const float *__restric
 #pragma unroll
             for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
             float den = 0.f;
-#pragma unroll 2
-            for (int k = k0; k < k1; ++k) {
-                const float2 ml = *reinterpret_cast<const float2 *>(part_ml + ((size_t)k * H + h) * 2);
-                const float wk = ml.x == -INFINITY ? 0.f : expf(ml.x - M);
-                den += wk * ml.y;
-                const float4 *po = reinterpret_cast<const float4 *>(part_o + ((size_t)k * H + h) * CK + 16 * lane);
-                const float4 *po0 = reinterpret_cast<const float4 *>(part_o + (((size_t)k * 64 + 2 * lane) * H + h) * 8);
-                const float4 *po1 = reinterpret_cast<const float4 *>(part_o + (((size_t)k * 64 + 2 * lane + 1) * H + h) * 8);
+            // Partials are merged in batches of KB whose loads are all issued before any is used,
+            // so a row with many chunks pays the memory latency once per batch, not per chunk.
+            constexpr int KB = 8;
+            for (int kb = k0; kb < k1; kb += KB) {
+                float4 v[KB][4];
+                float wk[KB];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 v = OCT ? (q < 2 ? po0[q] : po1[q - 2]) : po[q];
-                    acc4[q].x += wk * v.x;
-                    acc4[q].y += wk * v.y;
-                    acc4[q].z += wk * v.z;
-                    acc4[q].w += wk * v.w;
+                for (int u = 0; u < KB; ++u) {
+                    const int k = kb + u;
+                    wk[u] = 0.f;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) v[u][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (k < k1) {
+                        const float2 ml = *reinterpret_cast<const float2 *>(part_ml + ((size_t)k * H + h) * 2);
+                        wk[u] = ml.x == -INFINITY ? 0.f : expf(ml.x - M);
+                        den += wk[u] * ml.y;
+                        if (OCT) {
+                            const float4 *po0 = reinterpret_cast<const float4 *>(part_o + (((size_t)k * 64 + 2 * lane) * H + h) * 8);
+                            const float4 *po1 = reinterpret_cast<const float4 *>(part_o + (((size_t)k * 64 + 2 * lane + 1) * H + h) * 8);
+                            v[u][0] = po0[0];
+                            v[u][1] = po0[1];
+                            v[u][2] = po1[0];
+                            v[u][3] = po1[1];
+                        } else {
+                            const float4 *po = reinterpret_cast<const float4 *>(part_o + ((size_t)k * H + h) * CK + 16 * lane);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) v[u][q] = po[q];
+                        }
+                    }
                 }
+#pragma unroll
+                for (int u = 0; u < KB; ++u)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc4[q].x += wk[u] * v[u][q].x;
+                        acc4[q].y += wk[u] * v[u][q].y;
+                        acc4[q].z += wk[u] * v[u][q].z;
+                        acc4[q].w += wk[u] * v[u][q].w;
+                    }
             }
             const float inv = den > 0.f ? 1.f / den : 0.f;
 #pragma unroll

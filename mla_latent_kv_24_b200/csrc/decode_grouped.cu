@@ -53,14 +53,18 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
     float *red_ml = reinterpret_cast<float *>(gsm);                       // [WARPS][16][2], after the loop
     float *red_o = red_ml + WARPS * 16 * 2;                               // [WARPS][16][128], after the loop
 
-    const WorkItem it = p.plan.items[blockIdx.x];
-    const int g = blockIdx.y;
+    // blockIdx.x = group (fastest), so the 16 groups of a chunk run together and the chunk's RoPE
+    // keys, which every group reads, come from L2 after the first group's read.
+    const int item = blockIdx.z * 65535 + blockIdx.y;   // grid.y holds at most 65535 items
+    if (item >= p.plan.n_work) return;
+    const WorkItem it = p.plan.items[item];
+    const int g = blockIdx.x;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int b = it.row;                   // the plan of this path has one row per request
     const int L = p.seq_lens[b];
     const int G = p.H / GH;
     const int n_pg = ceil_div(it.t1 - it.t0, PAGE);
-    const size_t part_base = (size_t)blockIdx.x * p.s_q;
+    const size_t part_base = (size_t)item * p.s_q;
 
     if (it.t1 <= it.t0) {   // only in a rejected plan
         for (int i = tid; i < p.s_q * GH; i += blockDim.x) {
@@ -296,7 +300,7 @@ cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expa
         if (e != cudaSuccess) return e;
         attr = true;
     }
-    dim3 grid(plan.n_work, d.H / GH);
+    dim3 grid(d.H / GH, std::min(plan.n_work, 65535), ceil_div(plan.n_work, 65535));
     grouped_decode_kernel<<<grid, WARPS * 32, SMEM, st>>>(p);
     return cudaGetLastError();
 }
