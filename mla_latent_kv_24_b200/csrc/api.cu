@@ -341,13 +341,13 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
         else
             return fail(MLA_ERR_UNSUPPORTED, "tcgen05 partials need the tensor-core combine");
     } else {
+        MLA_CUDA(launch_q_rope(d, q, seq_lens, batch, s_q, qp, st), "launch q_rope");
         if (grouped_tc_ok(d)) {
             ProfileScope prof(st);
-            MLA_CUDA(launch_grouped_decode(d, q, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages, s_q,
-                                           part_o, part_ml, err, st),
+            MLA_CUDA(launch_grouped_decode(d, qp, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages,
+                                           s_q, part_o, part_ml, err, st),
                      "launch grouped decode");
         } else {
-            MLA_CUDA(launch_q_rope(d, q, seq_lens, batch, s_q, qp, st), "launch q_rope");
             ProfileScope prof(st);
             SimtDecodeArgs a{qp, latent, expanded, page_table, plan, max_pages, n_pages, s_q, 1, part_o, part_ml, err};
             MLA_CUDA(launch_decode_simt(d, a, st), "launch grouped decode (CUDA cores)");

@@ -36,11 +36,11 @@ static_assert(RED_BYTES <= STAGE_BYTES, "reduction buffer must fit in the stage 
 constexpr size_t SMEM = STAGE_BYTES + sizeof(__nv_bfloat16) * 16 * Q_LD;   // 92416 B: 2 CTAs per SM
 
 struct GParams {
-    const __nv_bfloat16 *q, *expanded, *latent;
+    const __nv_bfloat16 *q, *expanded, *latent;   // q: rotated queries [rows, H, 192]
     const int *page_table, *seq_lens;
     Plan plan;
     int max_pages, n_pages, s_q, H;
-    float scale_log2, base;
+    float scale_log2;
     float *part_o, *part_ml;   // [n_work * s_q, H, 128], [n_work * s_q, H, 2]
     int *err;
 };
@@ -74,24 +74,14 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
         }
         return;
     }
-    // Queries of this group: row m = j * 8 + hh (s_q = 2 fills all 16 rows, s_q = 1 the first 8).
-    for (int i = tid; i < 16 * (D_QK / 2); i += blockDim.x) {
-        const int m = i / (D_QK / 2), c = 2 * (i % (D_QK / 2));
+    // Queries of this group, already rotated (q_rot = [q_nope | RoPE(q_rope, p_j)], one pass per
+    // call): row m = j * 8 + hh; s_q = 2 fills all 16 rows, s_q = 1 the first 8 (rest zero).
+    for (int i = tid; i < 16 * (D_QK / 8); i += blockDim.x) {   // 16-byte chunks
+        const int m = i / (D_QK / 8), c = 8 * (i % (D_QK / 8));
         const int j = m / GH, h = g * GH + m % GH;
-        float x0 = 0.f, x1 = 0.f;
-        if (j < p.s_q) {
-            const __nv_bfloat16 *src = p.q + (((size_t)b * p.s_q + j) * p.H + h) * D_QK + c;
-            x0 = __bfloat162float(src[0]);
-            x1 = __bfloat162float(src[1]);
-            if (c >= D_N) {
-                float cs, sn;
-                rope_cos_sin(L - p.s_q + j, (c - D_N) / 2, D_R, p.base, &cs, &sn);
-                const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
-                x0 = y0;
-                x1 = y1;
-            }
-        }
-        *reinterpret_cast<uint32_t *>(qs + m * Q_LD + c) = pack_bf16(x0, x1);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (j < p.s_q) v = *reinterpret_cast<const uint4 *>(p.q + (((size_t)b * p.s_q + j) * p.H + h) * D_QK + c);
+        *reinterpret_cast<uint4 *>(qs + m * Q_LD + c) = v;
     }
     __syncthreads();
 
@@ -290,7 +280,6 @@ cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expa
     p.s_q = s_q;
     p.H = d.H;
     p.scale_log2 = d.scale * 1.4426950408889634f;
-    p.base = d.base;
     p.part_o = part_o;
     p.part_ml = part_ml;
     p.err = err;
