@@ -209,6 +209,20 @@ def oracle_sample(inp: wl.DecodeInputs, budget_s: float):
     return est, units, spent, desc
 
 
+# --------------------------------------------------------------------------- ranks
+def reduce_over_ranks(dist, device, times_ms, tokens):
+    """Whole-job figures of a weak-scaling run: the max over ranks of each device time (every rank
+    decodes its own batch; the job ends with the slowest) and the sum of the ranks' cache tokens
+    (ragged workloads draw different lengths per rank).  With dist None the run has one rank."""
+    import torch
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    n = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return t.tolist(), n.item()
+
+
 # --------------------------------------------------------------------------- GPU arm
 def run_ours(a, rank, world, local_rank):
     import torch
@@ -320,15 +334,12 @@ def run_ours(a, rank, world, local_rank):
         e2e = (e2e_ms, h_host.numel() * h_host.element_size() + q_host.numel() * q_host.element_size(),
                out_host.numel() * out_host.element_size())
 
-    t = torch.tensor([total_ms, kern_ms, e2e[0] if e2e else 0.0], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, kern_ms, e2e_ms = t.tolist()
+    (total_ms, kern_ms, e2e_ms), tokens_all = reduce_over_ranks(dist, dev, [total_ms, kern_ms, e2e[0] if e2e else 0.0],
+                                                                acct["tokens"])
 
     if rank == 0:
         peaks, peak_src = load_peaks()
         ms = total_ms / a.steps
-        tokens_all = acct["tokens"] * world
         value = tokens_all * a.steps / (total_ms / 1e3)
         kb, kf = acct["kernel_bytes"], acct["kernel_flops"]
         t_hbm = kb / (peaks["hbm_gbs"] * 1e9)
