@@ -26,7 +26,9 @@
  *     fp32 = IEEE float.  All pointers of one call use the dtype in dims->dtype, except int32
  *     index arrays.  Device pointers must be 16-byte aligned.
  *   - Positions: request b's cache holds seq_lens[b] tokens including its s_q current
- *     tokens; query j (0 <= j < s_q) sits at position seq_lens[b] - s_q + j and attends to
+ *     tokens (1 <= s_q <= 4: multi-token-prediction depth; the grouped tensor-core kernel
+ *     covers s_q <= 2, deeper s_q runs the CUDA-core grouped decode);
+ *     query j (0 <= j < s_q) sits at position seq_lens[b] - s_q + j and attends to
  *     tokens t <= that position (this gives the causal mask between MTP query tokens).
  *     Token t of request b lives in page page_table[b*max_pages + t/page_size], row
  *     t % page_size.
@@ -237,6 +239,43 @@ MLA_API mla_status mla_decode_absorbed_noalloc(const mla_dims *dims, const void 
  * changes.
  */
 MLA_API mla_status mla_set_profile_events(void *start_event, void *stop_event);
+
+/*
+ * mla_select_path — runtime choice between the two decoding paths of the same weights.
+ * ("GQLA ..." abstract: the runtime picks the path that matches the target hardware; the
+ *  MQA-absorb path trades memory traffic for computation and replicates the latent on every
+ *  rank, the GQA path shards its KV groups over up to 8 ranks.)  Pure host arithmetic: no
+ * CUDA call, no device pointer.
+ *
+ * Roofline model of one decode call on one rank (tp ranks share the heads):
+ *   visible  = sum_b sum_j (seq_lens[b] - s_q + j + 1)        (query-token pairs)
+ *   tokens   = sum_b seq_lens[b]
+ *   absorbed: bytes = tokens*(d_c + d_rope)*e            (the latent, replicated on every rank)
+ *                     + (G/tp)*(d_nope + d_v)*d_c*e           (this rank's W_UK and W_UV)
+ *             flops = visible*2*(H/tp)*(2*d_c + d_rope)
+ *                     + batch*s_q*(H/tp)*2*d_c*(d_nope + d_v)    (q absorption, W_UV)
+ *   grouped:  bytes = tokens*((G/tp)*(d_nope + d_v) + d_rope)*e
+ *             flops = visible*2*(H/tp)*(d_nope + d_rope + d_v)
+ *   time     = max(bytes / hbm_bytes_per_s, flops / flops_per_s) for each path
+ * with e the element size, G = H / heads_per_group, and q / out traffic left out (equal on
+ * both paths).  The grouped path's expanded cache must exist (gqla_expand_cache); its upkeep
+ * is per appended page and is not counted.
+ *
+ *   dims              as for the decode calls (heads_per_group = 8 for GQLA weights)
+ *   batch, s_q        > 0; 1 <= s_q <= 4
+ *   seq_lens_host     host [batch], each >= s_q
+ *   hbm_bytes_per_s   target memory bandwidth (> 0)
+ *   flops_per_s       target dense tensor throughput for dims->dtype (> 0)
+ *   tp                ranks that shard the heads / KV groups: 1 for one GPU; must divide
+ *                     H / heads_per_group
+ *   path              out: MLA_PATH_ABSORBED or MLA_PATH_GROUPED (the smaller time; absorbed
+ *                     on a tie)
+ *   t_absorbed_s, t_grouped_s   out (may be NULL): the two modelled times, seconds
+ */
+typedef enum { MLA_PATH_ABSORBED = 0, MLA_PATH_GROUPED = 1 } mla_path;
+MLA_API mla_status mla_select_path(const mla_dims *dims, int32_t batch, int32_t s_q, const int32_t *seq_lens_host,
+                                   double hbm_bytes_per_s, double flops_per_s, int32_t tp, mla_path *path,
+                                   double *t_absorbed_s, double *t_grouped_s);
 
 /* Text of the last error on the calling thread ("" if none).  Valid until the next call. */
 MLA_API const char *mla_last_error_string(void);

@@ -19,7 +19,7 @@ __all__ = [
     "mla_cache_append", "mla_decode_workspace_size", "mla_decode_absorbed",
     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
     "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
-    "mla_decode_absorbed_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
+    "mla_decode_absorbed_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS", "mla_select_path",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so")
@@ -31,7 +31,7 @@ MLA_BF16, MLA_FP32 = 0, 1
 EXPORTED_SYMBOLS = ["mla_cache_append", "mla_decode_workspace_size", "mla_decode_absorbed",
                     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
                     "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
-                    "mla_decode_absorbed_noalloc"]
+                    "mla_decode_absorbed_noalloc", "mla_select_path"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -81,6 +81,8 @@ def load() -> ctypes.CDLL:
         "mla_version": [],
         "mla_set_profile_events": [_P, _P],
         "mla_decode_absorbed_noalloc": [D, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P],
+        "mla_select_path": [D, _I, _I, _P, ctypes.c_double, ctypes.c_double, _I, ctypes.POINTER(ctypes.c_int),
+                            ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -193,3 +195,14 @@ def mla_decode_absorbed_noalloc(dims, q, W_uk, W_uv, latent_cache, page_table, s
     _check(load().mla_decode_absorbed_noalloc(ctypes.byref(dims), _dev(q), _dev(W_uk), _dev(W_uv), _dev(latent_cache),
                                               _dev(page_table), _dev(seq_lens), p, batch, s_q, max_pages,
                                               n_pages_total, _dev(out), _stream(stream)))
+
+
+def mla_select_path(dims, batch, s_q, seq_lens_host, hbm_bytes_per_s, flops_per_s, tp=1):
+    """Roofline choice between the two decoding paths (host arithmetic only, no GPU needed).
+    Returns ("absorbed" | "grouped", modelled seconds of the absorbed path, of the grouped path)."""
+    lens, lp = _host_i32(seq_lens_host)
+    path = ctypes.c_int(0)
+    ta, tg = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    _check(load().mla_select_path(ctypes.byref(dims), batch, s_q, lp, float(hbm_bytes_per_s), float(flops_per_s), tp,
+                                  ctypes.byref(path), ctypes.byref(ta), ctypes.byref(tg)))
+    return ("grouped" if path.value == 1 else "absorbed"), ta.value, tg.value

@@ -113,7 +113,7 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 
 mla_status check_batch(const Dims &d, int batch, int s_q, int max_pages, const int32_t *lens_host) {
     if (batch <= 0) return fail(MLA_ERR_INVALID_ARG, "batch must be > 0");
-    if (s_q < 1 || s_q > 2) return fail(MLA_ERR_INVALID_ARG, "s_q must be 1 or 2 (got %d)", s_q);
+    if (s_q < 1 || s_q > 4) return fail(MLA_ERR_INVALID_ARG, "s_q must be 1..4 (got %d)", s_q);
     if (max_pages <= 0) return fail(MLA_ERR_INVALID_ARG, "max_pages must be > 0");
     if (!lens_host) return fail(MLA_ERR_INVALID_ARG, "seq_lens_host is NULL");
     if ((long long)batch * s_q > (1 << 20)) return fail(MLA_ERR_UNSUPPORTED, "batch * s_q too large");
@@ -149,7 +149,7 @@ mla_status make_layout(const Dims &d, Path path, bool tc, int sms, int batch, in
     if (tc) {
         units = tc_units(sms);
         granule = tc_token_granule();
-    } else if (path == GROUPED && grouped_tc_ok(d)) {
+    } else if (path == GROUPED && grouped_tc_ok(d, s_q)) {
         units = grouped_units(d, sms);
         granule = grouped_token_granule();
     } else {
@@ -157,7 +157,7 @@ mla_status make_layout(const Dims &d, Path path, bool tc, int sms, int batch, in
         units = std::max(1, 4 * sms / std::max(1, d.H / hb));
         granule = 32;
     }
-    L->plan_sq = (path == GROUPED && grouped_tc_ok(d)) ? 1 : s_q;
+    L->plan_sq = (path == GROUPED && grouped_tc_ok(d, s_q)) ? 1 : s_q;
     L->qpi = s_q / L->plan_sq;
     L->chunk = plan_chunk(lens, batch, L->plan_sq, units, granule);
     L->n_work = (int)plan_count(lens, batch, L->plan_sq, L->chunk);
@@ -261,7 +261,7 @@ static mla_status decode_workspace(const mla_dims *dims, Path path, int32_t batc
     Dims d;
     MLA_TRY(check_dims(dims, &d));
     if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
-    if (batch <= 0 || s_q < 1 || s_q > 2 || !lens) return fail(MLA_ERR_INVALID_ARG, "bad batch / s_q / seq_lens_host");
+    if (batch <= 0 || s_q < 1 || s_q > 4 || !lens) return fail(MLA_ERR_INVALID_ARG, "bad batch / s_q / seq_lens_host");
     int sms = 0;
     MLA_TRY(device_info(nullptr, &sms));
     const bool tc = path == ABSORBED && use_tc_absorbed(dims);
@@ -342,7 +342,7 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
             return fail(MLA_ERR_UNSUPPORTED, "tcgen05 partials need the tensor-core combine");
     } else {
         MLA_CUDA(launch_q_rope(d, q, seq_lens, batch, s_q, qp, st), "launch q_rope");
-        if (grouped_tc_ok(d)) {
+        if (grouped_tc_ok(d, s_q)) {
             ProfileScope prof(st);
             MLA_CUDA(launch_grouped_decode(d, qp, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages,
                                            s_q, part_o, part_ml, err, st),
@@ -420,6 +420,37 @@ mla_status gqla_decode_grouped(const mla_dims *dims, const void *q, const void *
     return run_decode(GROUPED, dims, q, nullptr, nullptr, latent_cache, expanded_cache, page_table, seq_lens,
                       seq_lens_host, batch, s_q, max_pages, n_pages_total, out, workspace, workspace_bytes,
                       (cudaStream_t)stream);
+}
+
+mla_status mla_select_path(const mla_dims *dims, int32_t batch, int32_t s_q, const int32_t *seq_lens_host,
+                           double hbm_bytes_per_s, double flops_per_s, int32_t tp, mla_path *path,
+                           double *t_absorbed_s, double *t_grouped_s) {
+    g_last_error.clear();
+    Dims d;
+    MLA_TRY(check_dims(dims, &d));
+    if (!path) return fail(MLA_ERR_INVALID_ARG, "path is NULL");
+    if (batch <= 0 || s_q < 1 || s_q > 4 || !seq_lens_host) return fail(MLA_ERR_INVALID_ARG, "bad batch / s_q / seq_lens_host");
+    if (!(hbm_bytes_per_s > 0.0) || !(flops_per_s > 0.0)) return fail(MLA_ERR_INVALID_ARG, "peaks must be > 0");
+    const int G = d.n_groups();
+    if (tp < 1 || G % tp) return fail(MLA_ERR_INVALID_ARG, "tp = %d must divide the %d KV groups", tp, G);
+    double tokens = 0.0, visible = 0.0;
+    for (int b = 0; b < batch; ++b) {
+        const double L = seq_lens_host[b];
+        if (L < s_q) return fail(MLA_ERR_INVALID_ARG, "seq_lens_host[%d] = %d < s_q", b, seq_lens_host[b]);
+        tokens += L;
+        for (int j = 0; j < s_q; ++j) visible += L - s_q + j + 1;
+    }
+    const double e = (double)elt(d), heads = (double)d.H / tp, groups = (double)G / tp;
+    const double abs_bytes = tokens * (d.d_c + d.d_r) * e + groups * (d.d_n + d.d_v) * d.d_c * e;
+    const double abs_flops = visible * 2.0 * heads * (2.0 * d.d_c + d.d_r) + (double)batch * s_q * heads * 2.0 * d.d_c * (d.d_n + d.d_v);
+    const double grp_bytes = tokens * (groups * (d.d_n + d.d_v) + d.d_r) * e;
+    const double grp_flops = visible * 2.0 * heads * (d.d_n + d.d_r + d.d_v);
+    const double t_abs = std::max(abs_bytes / hbm_bytes_per_s, abs_flops / flops_per_s);
+    const double t_grp = std::max(grp_bytes / hbm_bytes_per_s, grp_flops / flops_per_s);
+    *path = t_grp < t_abs ? MLA_PATH_GROUPED : MLA_PATH_ABSORBED;
+    if (t_absorbed_s) *t_absorbed_s = t_abs;
+    if (t_grouped_s) *t_grouped_s = t_grp;
+    return MLA_OK;
 }
 
 mla_status gqla_expand_cache(const mla_dims *dims, const void *W_uk, const void *W_uv, const void *latent_cache,

@@ -257,8 +257,8 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
 
 }  // namespace
 
-bool grouped_tc_ok(const Dims &d) {
-    return d.bf16 && d.hpw == GH && d.d_n == D_N && d.d_v == D_V && d.d_r == D_R && d.d_c == D_LAT && d.page == PAGE &&
+bool grouped_tc_ok(const Dims &d, int s_q) {
+    return s_q <= 2 && d.bf16 && d.hpw == GH && d.d_n == D_N && d.d_v == D_V && d.d_r == D_R && d.d_c == D_LAT && d.page == PAGE &&
            d.H % GH == 0;
 }
 int grouped_units(const Dims &d, int sms) { return std::max(1, 8 * 2 * sms / std::max(1, d.H / GH)); }

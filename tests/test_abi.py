@@ -44,7 +44,7 @@ def test_invalid_arguments_return_status_without_device():
     assert _call_absorbed(mla.make_dims(heads_per_group=3)) == 1           # does not divide H
     assert _call_absorbed(mla.make_dims(d_c=1024)) == 2                    # unsupported dims
     assert _call_absorbed(mla.make_dims(page_size=48)) == 2
-    assert _call_absorbed(good, s_q=3, lens=(64,)) == 1                    # s_q out of range
+    assert _call_absorbed(good, s_q=5, lens=(64,)) == 1                    # s_q out of range (1..4)
     assert _call_absorbed(good, s_q=2, lens=(1,)) == 1                     # seq_len < s_q
     assert _call_absorbed(good, lens=(65,), max_pages=1) == 1              # seq_len > max_pages * page
     assert _call_absorbed(good, q=None) == 1                               # NULL pointer

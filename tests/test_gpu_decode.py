@@ -105,6 +105,25 @@ def test_grouped_ignores_nonfinite_stale_slots():
     assert_close(got, oracle_decode(inp), "bf16", "grouped with NaN stale slots")
 
 
+@pytest.mark.parametrize("s_q", [3, 4])
+def test_deeper_mtp_both_paths_match_oracle(s_q):
+    # s_q = 3, 4: the absorbed path decodes every query row; the grouped path runs its CUDA-core
+    # decode (its tensor-core tile holds two queries).  One request has exactly s_q tokens.
+    w = wl.small_workload(wl.WORKLOADS["5_8192_1"], B=3, s_q=s_q, lens=[s_q, 130, 700], shuffle_pages=True,
+                          seed=60 + s_q)
+    inp = wl.make_inputs(w)
+    dev = Dev(inp)
+    ref = oracle_decode(inp)
+    assert_close(wl.from_torch_f64(dev.decode_absorbed()), ref, "bf16", f"absorbed s_q={s_q}")
+    assert_close(wl.from_torch_f64(dev.decode_grouped(dev.expand())), ref, "bf16", f"grouped s_q={s_q}")
+
+
+def test_deeper_mtp_mla_weights_match_oracle():
+    w = wl.small_workload(wl.WORKLOADS["2"], B=2, s_q=4, lens=[4, 300], seed=64)
+    inp = wl.make_inputs(w)
+    assert_close(wl.from_torch_f64(Dev(inp).decode_absorbed()), oracle_decode(inp), "bf16", "MLA s_q=4")
+
+
 def test_expand_cache_matches_oracle():
     import oracle
     w = wl.small_workload(wl.WORKLOADS["5_8192_1"], B=2, lens=[100, 64], seed=5)
