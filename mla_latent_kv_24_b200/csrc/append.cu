@@ -225,7 +225,7 @@ cudaError_t launch_append_mma(const Dims &d, const void *h, int hidden, const vo
                               int max_pages, int n_pages, void *cache, int *err, cudaStream_t st) {
     const int ks = hidden / AP_SPLIT, ld = ks + 8;
     const size_t smem = sizeof(__nv_bfloat16) * (size_t)(AP_COLS + AP_TOK) * ld + sizeof(float) * AP_TOK * AP_COLS;
-    cudaError_t e = cudaFuncSetAttribute(append_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = raise_smem_limit((const void *)append_mma_kernel, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(9 * AP_SPLIT, ceil_div(n_tok, AP_TOK));
     append_mma_kernel<<<grid, 256, smem, st>>>((const __nv_bfloat16 *)h, hidden, (const __nv_bfloat16 *)W_dkv,

@@ -80,12 +80,14 @@ cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part
     const size_t smem = sizeof(float) * RB * DV;
     if (d.bf16) {
         auto k = combine_kernel<__nv_bfloat16>;
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = raise_smem_limit((const void *)k, smem);
+        if (e != cudaSuccess) return e;
         k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV, (const __nv_bfloat16 *)W_uv,
                                    d.hpw, d.d_v, (__nv_bfloat16 *)out);
     } else {
         auto k = combine_kernel<float>;
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = raise_smem_limit((const void *)k, smem);
+        if (e != cudaSuccess) return e;
         k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV, (const float *)W_uv, d.hpw, d.d_v,
                                    (float *)out);
     }
@@ -252,16 +254,10 @@ bool combine_mma_ok(const Dims &d, int DV, bool project) {
 cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
                                int rows, bool oct_layout, const void *W_uv, void *out, cudaStream_t st) {
     const size_t smem = sizeof(__nv_bfloat16) * ((size_t)CM * O_LD + 2 * (size_t)CN * W_LD);
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(combine_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(combine_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
     dim3 grid(d.H, ceil_div(rows, CM));
     auto k = oct_layout ? combine_mma_kernel<true> : combine_mma_kernel<false>;
+    cudaError_t e = raise_smem_limit((const void *)k, smem);
+    if (e != cudaSuccess) return e;
     k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, d.H, (const __nv_bfloat16 *)W_uv, d.hpw,
                                (__nv_bfloat16 *)out);
     return cudaGetLastError();

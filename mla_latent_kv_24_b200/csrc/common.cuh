@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "mla.h"
 
 namespace mla {
@@ -62,4 +64,35 @@ struct Plan {
     int chunk;
 };
 
+}  // namespace mla
+
+namespace mla {
+// Raises a kernel's dynamic shared-memory limit on the current device once, to the largest size
+// asked so far; later launches that need no more skip the driver call (it costs microseconds of
+// host time per launch).  Host only; thread-safe.
+inline cudaError_t raise_smem_limit(const void *kernel, size_t bytes) {
+    struct Entry {
+        const void *kernel;
+        int device;
+        size_t bytes;
+    };
+    static std::mutex mu;
+    static Entry table[256];
+    static int n = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    Entry *hit = nullptr;
+    for (int i = 0; i < n; ++i)
+        if (table[i].kernel == kernel && table[i].device == dev) hit = &table[i];
+    if (hit && hit->bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    if (hit)
+        hit->bytes = bytes;
+    else if (n < 256)
+        table[n++] = Entry{kernel, dev, bytes};
+    return cudaSuccess;
+}
 }  // namespace mla

@@ -283,12 +283,8 @@ cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expa
     p.part_o = part_o;
     p.part_ml = part_ml;
     p.err = err;
-    static bool attr = false;
-    if (!attr) {
-        cudaError_t e = cudaFuncSetAttribute(grouped_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
-        if (e != cudaSuccess) return e;
-        attr = true;
-    }
+    cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel, SMEM);
+    if (e != cudaSuccess) return e;
     dim3 grid(d.H / GH, std::min(plan.n_work, 65535), ceil_div(plan.n_work, 65535));
     grouped_decode_kernel<<<grid, WARPS * 32, SMEM, st>>>(p);
     return cudaGetLastError();

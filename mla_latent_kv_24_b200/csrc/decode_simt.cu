@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(P p) {
 template <typename T, int MODE>
 cudaError_t launch_t(const P &p, dim3 grid, size_t smem, cudaStream_t st) {
     auto k = decode_simt_kernel<T, MODE>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = raise_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
     k<<<grid, WARPS * 32, smem, st>>>(p);
     return cudaGetLastError();

@@ -543,6 +543,38 @@ bool encode_blocks(CUtensorMap *m, const void *ptr, uint64_t rows, int nblk, boo
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The maps depend only on (base pointer, rows, box shape); a decode loop passes the same buffers
+// every step, so recent encodings are reused (a host-side encoding costs about a microsecond).
+bool encode_blocks_cached(CUtensorMap *m, const void *ptr, uint64_t rows, int nblk, bool vsplit) {
+    struct Entry {
+        const void *ptr;
+        uint64_t rows;
+        int nblk, device;
+        bool vsplit;
+        CUtensorMap map;
+    };
+    static std::mutex mu;
+    static Entry cache[16];
+    static int used = 0, next = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (cache[i].ptr == ptr && cache[i].rows == rows && cache[i].nblk == nblk && cache[i].vsplit == vsplit &&
+                cache[i].device == dev) {
+                *m = cache[i].map;
+                return true;
+            }
+    }
+    if (!encode_blocks(m, ptr, rows, nblk, vsplit)) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    cache[next] = Entry{ptr, rows, nblk, dev, vsplit, *m};
+    next = (next + 1) % 16;
+    used = used < 16 ? used + 1 : 16;
+    return true;
+}
+
 }  // namespace
 
 bool tc_available() { return true; }
@@ -555,9 +587,9 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
     if (plan.n_work == 0) return cudaSuccess;
     CUtensorMap tm_q, tm_k, tm_page, tm_v;
     const uint64_t kv_rows = (uint64_t)n_pages * PAGE;
-    if (!encode_blocks(&tm_q, q_abs, (uint64_t)plan.rows * H, 9, false) ||
-        !encode_blocks(&tm_k, latent, kv_rows, 3, false) || !encode_blocks(&tm_page, latent, kv_rows, 9, false) ||
-        !encode_blocks(&tm_v, latent, kv_rows, 0, true))
+    if (!encode_blocks_cached(&tm_q, q_abs, (uint64_t)plan.rows * H, 9, false) ||
+        !encode_blocks_cached(&tm_k, latent, kv_rows, 3, false) ||
+        !encode_blocks_cached(&tm_page, latent, kv_rows, 9, false) || !encode_blocks_cached(&tm_v, latent, kv_rows, 0, true))
         return cudaErrorInvalidValue;
     TcParams p;
     p.plan = plan;
@@ -569,12 +601,8 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
     p.part_o = part_o;
     p.part_ml = part_ml;
     p.err = err;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(tc_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = raise_smem_limit((const void *)tc_decode_kernel, SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
     const int units = std::max(1, std::min(plan.n_work, std::max(1, sms / 2)));
     tc_decode_kernel<<<2 * units, THREADS, SMEM_ALLOC, st>>>(tm_q, tm_k, tm_page, tm_v, p);
     return cudaGetLastError();

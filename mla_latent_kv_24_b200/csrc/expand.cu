@@ -163,7 +163,8 @@ cudaError_t launch_expand(const Dims &d, const void *W_uk, const void *W_uv, con
     if (n_ids == 0) return cudaSuccess;
     if (d.bf16 && d.d_n == 128 && d.d_v == 128 && d.d_c % BK == 0) {
         const size_t smem = sizeof(__nv_bfloat16) * STAGES * (BM + BN) * LDS;
-        cudaFuncSetAttribute(expand_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = raise_smem_limit((const void *)expand_mma_kernel, smem);
+        if (e != cudaSuccess) return e;
         dim3 grid((unsigned)(((long long)n_ids * d.page + BM - 1) / BM), G, 2);
         expand_mma_kernel<<<grid, 256, smem, st>>>((const __nv_bfloat16 *)W_uk, (const __nv_bfloat16 *)W_uv,
                                                    (const __nv_bfloat16 *)latent, page_ids, n_ids, n_pages, d.page,
