@@ -5,8 +5,9 @@
 //     s_t = scale * ([q_nope | RoPE(q_rope, p_j)] . [K_g,t | k^R_t]),  t <= p_j
 //     o   = sum_t softmax(s)_t V_g,t
 //
-// The path is bound by HBM (8320 bytes per token for 16 groups, ~10 flop per byte per query),
-// so the kernel streams the expanded cache with deep cp.async pipelines and uses warp-level
+// The queries arrive rotated (the q RoPE kernel runs once per call).  The path is bound by HBM
+// (8320 bytes per token for 16 groups, ~10 flop per byte per query), so the kernel streams the
+// expanded cache through a two-stage cp.async pipeline, two CTAs per SM, and uses warp-level
 // mma.sync (m16n8k16, fp32 accumulators), whose throughput is far above what the bytes need.
 // One CTA takes one chunk of one request and one group: the group's 8 heads of every query of
 // the request form the 16 rows of the MMA tile (both MTP queries share each K/V tile), so each

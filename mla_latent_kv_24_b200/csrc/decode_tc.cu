@@ -28,9 +28,9 @@
 // 4-D views of the [rows, 576] cache whose inner dimensions are 64-column blocks): a single
 // thread issuing one small box at a time cannot reach HBM bandwidth, while one instruction per
 // 24-32 KiB can.  K and V have separate rings and producers, so a V slot held until its PV
-// never stalls the next step's K loads; the K producer also prefetches its pages into L2 three
-// steps ahead, so the shared-memory loads of a step see L2 rather than DRAM latency.  S is double-buffered in TMEM, so
-// QK^T of step g+1 runs while the softmax of step g works.  The softmax rescales O only when a
+// never stalls the next step's K loads.  (An L2 prefetch of the pages ahead of their K loads
+// was measured slower at every distance from one to four steps and is not used.)  S is
+// double-buffered in TMEM, so QK^T of step g+1 runs while the softmax of step g works.  The softmax rescales O only when a
 // row max grows by more than 2^8 (exact after the final division by l).  Every wait is bounded:
 // on timeout the kernel records MLA_ERR_TIMEOUT, stops issuing work, and still frees its
 // tensor memory before returning.
@@ -46,7 +46,6 @@ namespace {
 constexpr int H = 128, DROW = 576, PAGE = 64, STEP = 128;
 constexpr int NK = 3;                          // K ring: three slots of three 64-column blocks
 constexpr int NV = 2;                          // V ring: one slot per page of the step
-constexpr int PREFETCH_STEPS = 0;              // L2 prefetch distance of the K producer
 constexpr uint32_t BOX = 8192;                 // one 64-column block of 64 rows: 64 x 128 bytes
 constexpr uint32_t KSLOT = 3 * BOX;
 constexpr uint32_t VSLOT = 4 * BOX;            // [chunk 0..1][block pair][64 rows][64 cols]
@@ -146,13 +145,12 @@ __device__ __forceinline__ int page_row(const TcParams &p, int b, int pi, int t_
 // one 64-column block, the row dimension has stride 1152 B, the block dimension stride 128 B):
 //   tm_q    3-D (64, rows, 9),    box (64, 64, 9): 64 rows x 576 columns, block-major in smem
 //   tm_k    3-D (64, rows, 9),    box (64, 64, 3): 64 rows x three blocks
-//   tm_page same map with box (64, 64, 9), used for the L2 prefetch of a whole page
 //   tm_v    4-D (64, rows, 4, 2), strides (1152, 128, 512), box (64, 64, 2, 2): for chunk c in
 //           {0, 1} the two blocks starting at 4c + 2 rank, i.e. columns [256c + 128 rank, +128)
 // K producer: per work item the CTA's 64 query heads (Q), then per 128-token step the CTA's own
 // page of the step.  Steps are numbered across items (g), so every slot's phase is g's parity.
 __device__ void run_k_producer(const Ctx &c, const TcParams &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
-                               const CUtensorMap *tm_page, int pair, int n_pairs) {
+                               int pair, int n_pairs) {
     int g = 0, item_n = 0;
     for (int k = pair; k < p.plan.n_work; k += n_pairs) {
         const WorkItem it = p.plan.items[k];
@@ -160,17 +158,11 @@ __device__ void run_k_producer(const Ctx &c, const TcParams &p, const CUtensorMa
         const int b = it.row / p.s_q;
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
         auto own_row = [&](int i) { return page_row(p, b, (it.t0 + STEP * i) / PAGE + (int)c.rank, it.t1); };
-        auto prefetch = [&](int i) {
-            const int y = own_row(i);
-            if (y < p.n_pages * PAGE) tc::tma_prefetch_3d(tm_page, 0, y, 0);
-        };
-        for (int i = 0; i < PREFETCH_STEPS && i < n_steps; ++i) prefetch(i);
         if (item_n > 0 && !wait_or_abort(c, c.bar(B_QEMPTY), (uint32_t)(item_n - 1) & 1u, p.err)) return;
         ++item_n;
         if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_QFULL), 2u * Q_BYTES);
         tc::tma_load_3d_pair(c.base + OFF_Q, tm_q, 0, it.row * H + 64 * (int)c.rank, 0, c.lead_bar(B_QFULL));
         for (int i = 0; i < n_steps; ++i, ++g) {
-            if (i + PREFETCH_STEPS < n_steps) prefetch(i + PREFETCH_STEPS);
             const int y = own_row(i);
             for (int j = 0; j < NK; ++j) {
                 if (!wait_or_abort(c, c.bar(B_KEMPTY + j), ((uint32_t)g & 1u) ^ 1u, p.err)) return;
@@ -423,7 +415,7 @@ __device__ void run_softmax(const Ctx &c, const TcParams &p, uint32_t tmem, int 
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_page, const __grid_constant__ CUtensorMap tm_v, TcParams p) {
+                     const __grid_constant__ CUtensorMap tm_v, TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     Ctx c;
     const uint32_t raw = tc::smem_addr(smem_raw);
@@ -463,7 +455,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     if (warp == W_KPROD && lane == 0) {
         tc::prefetch_tmap(&tm_q);
         tc::prefetch_tmap(&tm_k);
-        tc::prefetch_tmap(&tm_page);
         tc::prefetch_tmap(&tm_v);
     }
     if (warp == W_MMA) tc::tmem_alloc_pair(c.base + OFF_TMEMPTR, TM_COLS);
@@ -475,7 +466,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     const int pair = blockIdx.x / 2, n_pairs = gridDim.x / 2;
     if (warp == W_KPROD) {
-        if (lane == 0) run_k_producer(c, p, &tm_q, &tm_k, &tm_page, pair, n_pairs);
+        if (lane == 0) run_k_producer(c, p, &tm_q, &tm_k, pair, n_pairs);
     } else if (warp == W_VPROD) {
         if (lane == 0) run_v_producer(c, p, &tm_v, pair, n_pairs);
     } else if (warp == W_MMA) {
@@ -585,11 +576,10 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
                              const Plan &plan, int max_pages, int n_pages, int s_q, float *part_o, float *part_ml,
                              int *err, int sms, cudaStream_t st) {
     if (plan.n_work == 0) return cudaSuccess;
-    CUtensorMap tm_q, tm_k, tm_page, tm_v;
+    CUtensorMap tm_q, tm_k, tm_v;
     const uint64_t kv_rows = (uint64_t)n_pages * PAGE;
     if (!encode_blocks_cached(&tm_q, q_abs, (uint64_t)plan.rows * H, 9, false) ||
-        !encode_blocks_cached(&tm_k, latent, kv_rows, 3, false) ||
-        !encode_blocks_cached(&tm_page, latent, kv_rows, 9, false) || !encode_blocks_cached(&tm_v, latent, kv_rows, 0, true))
+        !encode_blocks_cached(&tm_k, latent, kv_rows, 3, false) || !encode_blocks_cached(&tm_v, latent, kv_rows, 0, true))
         return cudaErrorInvalidValue;
     TcParams p;
     p.plan = plan;
@@ -604,7 +594,7 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
     cudaError_t e = raise_smem_limit((const void *)tc_decode_kernel, SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     const int units = std::max(1, std::min(plan.n_work, std::max(1, sms / 2)));
-    tc_decode_kernel<<<2 * units, THREADS, SMEM_ALLOC, st>>>(tm_q, tm_k, tm_page, tm_v, p);
+    tc_decode_kernel<<<2 * units, THREADS, SMEM_ALLOC, st>>>(tm_q, tm_k, tm_v, p);
     return cudaGetLastError();
 }
 
