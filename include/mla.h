@@ -241,6 +241,35 @@ MLA_API mla_status mla_decode_absorbed_noalloc(const mla_dims *dims, const void 
 MLA_API mla_status mla_set_profile_events(void *start_event, void *stop_event);
 
 /*
+ * mla_prefill_workspace_size / mla_prefill_expanded — head-expanded causal attention of the last
+ * n_q tokens of every request: a prefill chunk, or a batch of n_q draft tokens to verify.
+ * ("GQLA ..." abstract: MLA offers absorbed and head-expanded forms; the expanded form attends
+ *  with keys and values up-projected per head, "MLA and GRPO architecture", "The Mathematics
+ *  of MLA": k^C = W_UK c, v^C = W_UV c.)  For head h in group g = h / heads_per_group and query
+ * j at position p_j = seq_lens[b] - n_q + j:
+ *     s_t = scale * ([q_nope | RoPE(q_rope, p_j)] . [K_g,t | k^R_t]),  t <= p_j
+ *     out = sum_t softmax(s)_t V_g,t
+ * with K_g, V_g the expanded cache of gqla_expand_cache (pass dims with heads_per_group = 1
+ * there for per-head MLA weights).  Same math as gqla_decode_grouped, for any n_q.
+ *
+ *   q             device [batch, n_q, H, d_nope + d_rope]; RoPE part NOT yet rotated.
+ *   expanded_cache device [n_pages_total, H / heads_per_group, page_size, d_nope + d_v].
+ *   latent_cache  device [n_pages_total, page_size, d_c + d_rope] (source of k^R).
+ *   page_table, seq_lens, seq_lens_host as for the decode calls, with n_q <= seq_lens[b].
+ *   out           device [batch, n_q, H, d_v].
+ *   workspace     >= mla_prefill_workspace_size() bytes, 256-byte aligned (scratch).
+ * Needs bf16, d_nope = d_v = 128, d_rope = 64, d_c = 512, page_size = 64
+ * (MLA_ERR_UNSUPPORTED otherwise).
+ */
+MLA_API mla_status mla_prefill_workspace_size(const mla_dims *dims, int32_t batch, int32_t n_q,
+                                              const int32_t *seq_lens_host, size_t *bytes);
+MLA_API mla_status mla_prefill_expanded(const mla_dims *dims, const void *q, const void *expanded_cache,
+                                        const void *latent_cache, const int32_t *page_table, const int32_t *seq_lens,
+                                        const int32_t *seq_lens_host, int32_t batch, int32_t n_q, int32_t max_pages,
+                                        int32_t n_pages_total, void *out, void *workspace, size_t workspace_bytes,
+                                        mla_stream_t stream);
+
+/*
  * mla_select_path — runtime choice between the two decoding paths of the same weights.
  * ("GQLA ..." abstract: the runtime picks the path that matches the target hardware; the
  *  MQA-absorb path trades memory traffic for computation and replicates the latent on every

@@ -20,6 +20,7 @@ __all__ = [
     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
     "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
     "mla_decode_absorbed_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS", "mla_select_path",
+    "mla_prefill_workspace_size", "mla_prefill_expanded",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so")
@@ -31,7 +32,8 @@ MLA_BF16, MLA_FP32 = 0, 1
 EXPORTED_SYMBOLS = ["mla_cache_append", "mla_decode_workspace_size", "mla_decode_absorbed",
                     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
                     "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
-                    "mla_decode_absorbed_noalloc", "mla_select_path"]
+                    "mla_decode_absorbed_noalloc", "mla_select_path", "mla_prefill_workspace_size",
+                    "mla_prefill_expanded"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -83,6 +85,8 @@ def load() -> ctypes.CDLL:
         "mla_decode_absorbed_noalloc": [D, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P],
         "mla_select_path": [D, _I, _I, _P, ctypes.c_double, ctypes.c_double, _I, ctypes.POINTER(ctypes.c_int),
                             ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)],
+        "mla_prefill_workspace_size": [D, _I, _I, _P, ctypes.POINTER(_S)],
+        "mla_prefill_expanded": [D, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _S, _P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -206,3 +210,19 @@ def mla_select_path(dims, batch, s_q, seq_lens_host, hbm_bytes_per_s, flops_per_
     _check(load().mla_select_path(ctypes.byref(dims), batch, s_q, lp, float(hbm_bytes_per_s), float(flops_per_s), tp,
                                   ctypes.byref(path), ctypes.byref(ta), ctypes.byref(tg)))
     return ("grouped" if path.value == 1 else "absorbed"), ta.value, tg.value
+
+
+def mla_prefill_workspace_size(dims, batch, n_q, seq_lens_host) -> int:
+    arr, p = _host_i32(seq_lens_host)
+    n = _S(0)
+    _check(load().mla_prefill_workspace_size(ctypes.byref(dims), batch, n_q, p, ctypes.byref(n)))
+    return n.value
+
+
+def mla_prefill_expanded(dims, q, expanded_cache, latent_cache, page_table, seq_lens, seq_lens_host, batch, n_q,
+                         max_pages, n_pages_total, out, workspace, workspace_bytes=None, stream=None) -> None:
+    arr, p = _host_i32(seq_lens_host)
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(load().mla_prefill_expanded(ctypes.byref(dims), _dev(q), _dev(expanded_cache), _dev(latent_cache),
+                                       _dev(page_table), _dev(seq_lens), p, batch, n_q, max_pages, n_pages_total,
+                                       _dev(out), _dev(workspace), nbytes, _stream(stream)))

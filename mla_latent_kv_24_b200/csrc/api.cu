@@ -422,6 +422,96 @@ mla_status gqla_decode_grouped(const mla_dims *dims, const void *q, const void *
                       (cudaStream_t)stream);
 }
 
+// Prefill layout: q_rot [batch*n_q, H, 192] bf16 | one work item per request | row starts |
+// partial O [batch*n_q, H, d_v] fp32 | (m, l) [batch*n_q, H, 2].  One item per request: the
+// (head, 16-query tile) CTAs already fill the GPU, and one partial per query keeps the scratch
+// linear in n_q.
+static mla_status prefill_layout(const mla_dims *dims, int32_t batch, int32_t n_q, const int32_t *lens, Dims *d,
+                                 Layout *L) {
+    MLA_TRY(check_dims(dims, d));
+    if (!prefill_ok(*d)) return fail(MLA_ERR_UNSUPPORTED, "prefill needs bf16, d_nope = d_v = 128, d_rope = 64, d_c = 512, page 64");
+    if (batch <= 0 || n_q < 1 || !lens) return fail(MLA_ERR_INVALID_ARG, "bad batch / n_q / seq_lens_host");
+    if ((long long)batch * n_q > (1 << 20)) return fail(MLA_ERR_UNSUPPORTED, "batch * n_q too large");
+    long long longest = 1;
+    for (int b = 0; b < batch; ++b) {
+        if (lens[b] < n_q) return fail(MLA_ERR_INVALID_ARG, "seq_lens[%d] = %d < n_q = %d", b, lens[b], n_q);
+        longest = std::max<long long>(longest, lens[b]);
+    }
+    L->rows = batch * n_q;
+    L->plan_sq = 1;
+    L->qpi = n_q;
+    L->DK = d->d_n + d->d_r;
+    L->DV = d->d_v;
+    L->tc = false;
+    L->chunk = (int)((longest + d->page - 1) / d->page * d->page);
+    L->n_work = batch;
+    size_t off = 0;
+    L->q_off = off;
+    off = align256(off + (size_t)L->rows * d->H * L->DK * elt(*d));
+    L->items_off = off;
+    off = align256(off + (size_t)L->n_work * sizeof(WorkItem));
+    L->row_off = off;
+    off = align256(off + (size_t)(batch + 1) * sizeof(int));
+    L->po_off = off;
+    off = align256(off + (size_t)L->rows * d->H * L->DV * sizeof(float));
+    L->pml_off = off;
+    off = align256(off + (size_t)L->rows * d->H * 2 * sizeof(float));
+    L->total = off;
+    return MLA_OK;
+}
+
+mla_status mla_prefill_workspace_size(const mla_dims *dims, int32_t batch, int32_t n_q, const int32_t *seq_lens_host,
+                                      size_t *bytes) {
+    g_last_error.clear();
+    if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
+    Dims d;
+    Layout L;
+    MLA_TRY(prefill_layout(dims, batch, n_q, seq_lens_host, &d, &L));
+    *bytes = L.total;
+    return MLA_OK;
+}
+
+mla_status mla_prefill_expanded(const mla_dims *dims, const void *q, const void *expanded_cache,
+                                const void *latent_cache, const int32_t *page_table, const int32_t *seq_lens,
+                                const int32_t *seq_lens_host, int32_t batch, int32_t n_q, int32_t max_pages,
+                                int32_t n_pages_total, void *out, void *workspace, size_t workspace_bytes,
+                                mla_stream_t stream) {
+    g_last_error.clear();
+    Dims d;
+    Layout L;
+    MLA_TRY(prefill_layout(dims, batch, n_q, seq_lens_host, &d, &L));
+    if (max_pages <= 0 || n_pages_total <= 0) return fail(MLA_ERR_INVALID_ARG, "max_pages and n_pages_total must be > 0");
+    for (int b = 0; b < batch; ++b)
+        if ((long long)seq_lens_host[b] > (long long)max_pages * d.page)
+            return fail(MLA_ERR_INVALID_ARG, "seq_lens[%d] = %d > max_pages * page", b, seq_lens_host[b]);
+    if (!q || !expanded_cache || !latent_cache || !page_table || !seq_lens || !out)
+        return fail(MLA_ERR_INVALID_ARG, "NULL device pointer");
+    if (!aligned16(q) || !aligned16(expanded_cache) || !aligned16(latent_cache) || !aligned16(out))
+        return fail(MLA_ERR_INVALID_ARG, "device tensors must be 16-byte aligned");
+    MLA_TRY(check_ws(L, workspace, workspace_bytes));
+    int *err = nullptr;
+    MLA_TRY(device_info(&err, nullptr));
+    cudaStream_t st = (cudaStream_t)stream;
+    char *w = (char *)workspace;
+    WorkItem *items = (WorkItem *)(w + L.items_off);
+    int *row_first = (int *)(w + L.row_off);
+    float *part_o = (float *)(w + L.po_off);
+    float *part_ml = (float *)(w + L.pml_off);
+    void *qp = w + L.q_off;
+    Plan plan{items, row_first, L.n_work, batch, L.chunk};
+    MLA_CUDA(launch_plan(seq_lens, batch, 1, max_pages, d.page, L.chunk, L.n_work, items, row_first, err, st),
+             "launch plan");
+    MLA_CUDA(launch_q_rope(d, q, seq_lens, batch, n_q, qp, st), "launch q_rope");
+    {
+        ProfileScope prof(st);
+        MLA_CUDA(launch_prefill_expanded(d, qp, expanded_cache, latent_cache, seq_lens, page_table, plan, max_pages,
+                                         n_pages_total, n_q, part_o, part_ml, err, st),
+                 "launch prefill");
+    }
+    MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, n_q, L.DV, nullptr, out, st), "launch combine");
+    return MLA_OK;
+}
+
 mla_status mla_select_path(const mla_dims *dims, int32_t batch, int32_t s_q, const int32_t *seq_lens_host,
                            double hbm_bytes_per_s, double flops_per_s, int32_t tp, mla_path *path,
                            double *t_absorbed_s, double *t_grouped_s) {

@@ -14,6 +14,12 @@
 // page of K_g|V_g (32 KiB, contiguous) and of k^R (8 KiB) is read once per chunk.  Four warps
 // each take 16 tokens of every 64-token page and keep their own online softmax; the CTA merges
 // the four (m, l, O) at the end and writes one partial result per query for the combine.
+//
+// The same kernel serves the head-expanded prefill path ("GQLA ..." abstract: MLA's absorbed
+// and head-expanded forms; the expanded form attends with K and V up-projected per head):
+// PREFILL CTAs take one head and 16 consecutive query tokens of a request (rows = queries),
+// read the per-head (heads_per_group = 1) or per-group expanded cache, and skip the pages that
+// lie after their last query's position (causal).
 #include <math.h>
 
 #include "tc_decode.h"
@@ -40,12 +46,15 @@ struct GParams {
     const __nv_bfloat16 *q, *expanded, *latent;   // q: rotated queries [rows, H, 192]
     const int *page_table, *seq_lens;
     Plan plan;
-    int max_pages, n_pages, s_q, H;
+    int max_pages, n_pages, s_q, H, hpw;          // s_q: queries per request (prefill: n_q)
     float scale_log2;
     float *part_o, *part_ml;   // [n_work * s_q, H, 128], [n_work * s_q, H, 2]
     int *err;
 };
 
+// Rows of the MMA tile.  Decode: CTA = (group g, item), row m = query m / 8 of head g*8 + m % 8.
+// Prefill: CTA = (head, item, query tile), row m = query 16 * tile + m of that head.
+template <bool PREFILL>
 __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p) {
     extern __shared__ __align__(16) uint8_t gsm[];
     __nv_bfloat16 *kv = reinterpret_cast<__nv_bfloat16 *>(gsm);           // [STAGES][64][KV_LD]
@@ -56,30 +65,38 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
 
     // blockIdx.x = group (fastest), so the 16 groups of a chunk run together and the chunk's RoPE
     // keys, which every group reads, come from L2 after the first group's read.
-    const int item = blockIdx.z * 65535 + blockIdx.y;   // grid.y holds at most 65535 items
+    const int item = PREFILL ? (int)blockIdx.y : (int)(blockIdx.z * 65535 + blockIdx.y);   // grid.y <= 65535
     if (item >= p.plan.n_work) return;
     const WorkItem it = p.plan.items[item];
-    const int g = blockIdx.x;
+    const int tile = PREFILL ? (int)blockIdx.z : 0;
+    const int head = blockIdx.x;                                  // prefill: the CTA's head
+    const int g = PREFILL ? head / p.hpw : (int)blockIdx.x;       // expanded-cache group
+    const int G = PREFILL ? p.H / p.hpw : p.H / GH;
+    auto row_query = [&](int m) { return PREFILL ? 16 * tile + m : m / GH; };
+    auto row_head = [&](int m) { return PREFILL ? head : g * GH + m % GH; };
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int b = it.row;                   // the plan of this path has one row per request
     const int L = p.seq_lens[b];
-    const int G = p.H / GH;
-    const int n_pg = ceil_div(it.t1 - it.t0, PAGE);
+    // Pages after the tile's last query position are fully masked and are not read.
+    const int last_q = min(p.s_q, row_query(15) + 1) - 1;
+    const int t_end = min(it.t1, L - p.s_q + last_q + 1);
+    const int n_pg = t_end > it.t0 ? ceil_div(t_end - it.t0, PAGE) : 0;
     const size_t part_base = (size_t)item * p.s_q;
 
     if (it.t1 <= it.t0) {   // only in a rejected plan
-        for (int i = tid; i < p.s_q * GH; i += blockDim.x) {
-            const size_t r = part_base + i / GH;
-            p.part_ml[(r * p.H + g * GH + i % GH) * 2] = -INFINITY;
-            p.part_ml[(r * p.H + g * GH + i % GH) * 2 + 1] = 0.f;
+        for (int m = tid; m < 16; m += blockDim.x) {
+            if (row_query(m) >= p.s_q) continue;
+            const size_t r = part_base + row_query(m);
+            p.part_ml[(r * p.H + row_head(m)) * 2] = -INFINITY;
+            p.part_ml[(r * p.H + row_head(m)) * 2 + 1] = 0.f;
         }
         return;
     }
-    // Queries of this group, already rotated (q_rot = [q_nope | RoPE(q_rope, p_j)], one pass per
-    // call): row m = j * 8 + hh; s_q = 2 fills all 16 rows, s_q = 1 the first 8 (rest zero).
+    // Queries, already rotated (q_rot = [q_nope | RoPE(q_rope, p_j)], one pass per call).  Decode:
+    // s_q = 2 fills all 16 rows, s_q = 1 the first 8; rows past the last query are zero.
     for (int i = tid; i < 16 * (D_QK / 8); i += blockDim.x) {   // 16-byte chunks
         const int m = i / (D_QK / 8), c = 8 * (i % (D_QK / 8));
-        const int j = m / GH, h = g * GH + m % GH;
+        const int j = row_query(m), h = row_head(m);
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (j < p.s_q) v = *reinterpret_cast<const uint4 *>(p.q + (((size_t)b * p.s_q + j) * p.H + h) * D_QK + c);
         *reinterpret_cast<uint4 *>(qs + m * Q_LD + c) = v;
@@ -120,14 +137,14 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
 
     const int gid = lane / 4, t4 = lane % 4;
     // Rows gid and gid + 8 of this thread's fragments: query index and visible length.
-    const int lim0 = (gid / GH < p.s_q) ? L - p.s_q + gid / GH : -1;            // rows 0..7: query 0
-    const int lim1 = ((gid + 8) / GH < p.s_q) ? L - p.s_q + (gid + 8) / GH : -1; // rows 8..15: query 1
+    const int lim0 = row_query(gid) < p.s_q ? L - p.s_q + row_query(gid) : -1;
+    const int lim1 = row_query(gid + 8) < p.s_q ? L - p.s_q + row_query(gid + 8) : -1;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     float o[16][4];
 #pragma unroll
     for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
 
-    load_page(0, 0);
+    if (n_pg > 0) load_page(0, 0);
     cp_async_commit();
     for (int i = 0; i < n_pg; ++i) {
         if (i + 1 < n_pg) load_page((i + 1) % STAGES, i + 1);
@@ -231,9 +248,9 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
         red_o[(warp * 16 + gid + 8) * D_V + 8 * n + 2 * t4 + 1] = o[n][3];
     }
     __syncthreads();
-    // 16 rows x 128 columns; rows past s_q * 8 are padding.
+    // 16 rows x 128 columns; rows past the last query are padding.
     for (int i = tid; i < 16 * D_V; i += blockDim.x) {
-        const int m = i / D_V, c = i % D_V, j = m / GH;
+        const int m = i / D_V, c = i % D_V, j = row_query(m);
         if (j >= p.s_q) continue;
         float M = -INFINITY;
 #pragma unroll
@@ -247,7 +264,7 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
             den += wt * red_ml[(w * 16 + m) * 2 + 1];
         }
         const size_t r = part_base + j;
-        const int h = g * GH + m % GH;
+        const int h = row_head(m);
         p.part_o[(r * p.H + h) * D_V + c] = num;   // relative to max M (log2 units)
         if (c == 0) {
             p.part_ml[(r * p.H + h) * 2] = M * 0.69314718055994531f;
@@ -265,10 +282,9 @@ bool grouped_tc_ok(const Dims &d, int s_q) {
 int grouped_units(const Dims &d, int sms) { return std::max(1, 8 * 2 * sms / std::max(1, d.H / GH)); }
 int grouped_token_granule() { return PAGE; }
 
-cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expanded, const void *latent,
-                                  const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
-                                  int n_pages, int s_q, float *part_o, float *part_ml, int *err, cudaStream_t st) {
-    if (plan.n_work == 0) return cudaSuccess;
+static GParams grouped_params(const Dims &d, const void *q, const void *expanded, const void *latent,
+                              const int *seq_lens, const int *page_table, const Plan &plan, int max_pages, int n_pages,
+                              int s_q, float *part_o, float *part_ml, int *err) {
     GParams p;
     p.q = (const __nv_bfloat16 *)q;
     p.expanded = (const __nv_bfloat16 *)expanded;
@@ -280,14 +296,42 @@ cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expa
     p.n_pages = n_pages;
     p.s_q = s_q;
     p.H = d.H;
+    p.hpw = d.hpw;
     p.scale_log2 = d.scale * 1.4426950408889634f;
     p.part_o = part_o;
     p.part_ml = part_ml;
     p.err = err;
-    cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel, SMEM);
+    return p;
+}
+
+cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expanded, const void *latent,
+                                  const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
+                                  int n_pages, int s_q, float *part_o, float *part_ml, int *err, cudaStream_t st) {
+    if (plan.n_work == 0) return cudaSuccess;
+    const GParams p = grouped_params(d, q, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages, s_q,
+                                     part_o, part_ml, err);
+    cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<false>, SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(d.H / GH, std::min(plan.n_work, 65535), ceil_div(plan.n_work, 65535));
-    grouped_decode_kernel<<<grid, WARPS * 32, SMEM, st>>>(p);
+    grouped_decode_kernel<false><<<grid, WARPS * 32, SMEM, st>>>(p);
+    return cudaGetLastError();
+}
+
+bool prefill_ok(const Dims &d) {
+    return d.bf16 && d.d_n == D_N && d.d_v == D_V && d.d_r == D_R && d.d_c == D_LAT && d.page == PAGE;
+}
+
+cudaError_t launch_prefill_expanded(const Dims &d, const void *q_rot, const void *expanded, const void *latent,
+                                    const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
+                                    int n_pages, int n_q, float *part_o, float *part_ml, int *err, cudaStream_t st) {
+    if (plan.n_work == 0) return cudaSuccess;
+    if (plan.n_work > 65535 || ceil_div(n_q, 16) > 65535) return cudaErrorInvalidValue;
+    const GParams p = grouped_params(d, q_rot, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages, n_q,
+                                     part_o, part_ml, err);
+    cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<true>, SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid(d.H, plan.n_work, ceil_div(n_q, 16));
+    grouped_decode_kernel<true><<<grid, WARPS * 32, SMEM, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -18,6 +18,13 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
 bool grouped_tc_ok(const Dims &d, int s_q);   // s_q <= 2: one 16-row tile = 8 heads x 2 queries
 int grouped_units(const Dims &d, int sms);
 int grouped_token_granule();
+// Head-expanded prefill over the expanded cache (per head with heads_per_group = 1, or per
+// group): bf16, d_nope = d_v = 128, d_rope = 64, d_c = 512, page 64.  n_q query tokens per
+// request (the last n_q positions), partials [n_work * n_q, H, 128] for the combine.
+bool prefill_ok(const Dims &d);
+cudaError_t launch_prefill_expanded(const Dims &d, const void *q_rot, const void *expanded, const void *latent,
+                                    const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
+                                    int n_pages, int n_q, float *part_o, float *part_ml, int *err, cudaStream_t st);
 cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expanded, const void *latent,
                                   const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
                                   int n_pages, int s_q, float *part_o, float *part_ml, int *err, cudaStream_t st);

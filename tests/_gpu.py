@@ -59,6 +59,17 @@ class Dev:
         return out
 
 
+def prefill(dev: "Dev", expanded):
+    """Head-expanded prefill of the workload's last s_q tokens (n_q = s_q) through the C ABI."""
+    w = dev.inp.w
+    nb = mla.mla_prefill_workspace_size(dev.dims, w.B, w.s_q, dev.inp.seq_lens)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev.q.device)
+    out = torch.empty((w.B, w.s_q, w.H, w.d_v), dtype=dev.tdtype, device=dev.q.device)
+    mla.mla_prefill_expanded(dev.dims, dev.q, expanded, dev.cache, dev.page_table, dev.seq_lens, dev.inp.seq_lens,
+                             w.B, w.s_q, dev.max_pages, dev.inp.n_pages, out, ws)
+    return out
+
+
 def errors(got: np.ndarray, ref: np.ndarray):
     """(normwise max relative error, mean absolute error) over the finite entries of ref."""
     m = np.isfinite(ref)

@@ -70,3 +70,18 @@ def test_binding_raises_mla_error():
     with pytest.raises(mla.MlaError) as e:
         mla.mla_decode_workspace_size(d, 1, 1, [64])
     assert e.value.status == 1
+
+
+def test_prefill_argument_checks_without_device():
+    import mla_latent_kv_24_b200 as mla
+    dims = mla.make_dims()
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_prefill_workspace_size(dims, 2, 300, [100, 500])          # n_q > seq_len
+    assert e.value.status == 1
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_prefill_workspace_size(mla.make_dims(dtype="fp32"), 1, 4, [64])   # not built for fp32
+    assert e.value.status == 2
+    # scratch is linear in n_q: q_rot + partials + (m, l) per query row, one work item per request
+    a = mla.mla_prefill_workspace_size(dims, 2, 16, [100, 500])
+    b = mla.mla_prefill_workspace_size(dims, 2, 32, [100, 500])
+    assert 1.9 < b / a < 2.1
