@@ -77,10 +77,11 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int b = it.row;                   // the plan of this path has one row per request
     const int L = p.seq_lens[b];
-    // Pages after the tile's last query position are fully masked and are not read.
+    // Prefill: pages after the tile's last query position are fully masked and are not read.
+    // Decode: every chunk ends at or before L, which the last query sees, so all its pages count.
     const int last_q = min(p.s_q, row_query(15) + 1) - 1;
-    const int t_end = min(it.t1, L - p.s_q + last_q + 1);
-    const int n_pg = t_end > it.t0 ? ceil_div(t_end - it.t0, PAGE) : 0;
+    const int t_end = PREFILL ? min(it.t1, L - p.s_q + last_q + 1) : it.t1;
+    const int n_pg = PREFILL ? (t_end > it.t0 ? ceil_div(t_end - it.t0, PAGE) : 0) : ceil_div(it.t1 - it.t0, PAGE);
     const size_t part_base = (size_t)item * p.s_q;
 
     if (it.t1 <= it.t0) {   // only in a rejected plan
@@ -144,7 +145,7 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
 #pragma unroll
     for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
 
-    if (n_pg > 0) load_page(0, 0);
+    if (!PREFILL || n_pg > 0) load_page(0, 0);
     cp_async_commit();
     for (int i = 0; i < n_pg; ++i) {
         if (i + 1 < n_pg) load_page((i + 1) % STAGES, i + 1);
