@@ -83,8 +83,11 @@ def algorithmic(w: wl.Workload, lens: np.ndarray, path: str):
         G = w.n_w
         k_bytes = tokens * (G * (w.d_n + w.d_v) + w.d_r) * e + rows * w.H * w.d_qk * e
         k_flops = visible * 2 * w.H * (w.d_qk + w.d_v)
-        step_bytes = k_bytes + rows * w.H * w.d_v * e + w.d_row * w.hidden * e + rows * w.hidden * e
-        step_flops = k_flops + rows * 2 * w.d_row * w.hidden
+        # + the new tokens' expansion: W_UK and W_UV read, their latent rows read, [K_g | V_g] written
+        expand_bytes = (G * w.d_c * (w.d_n + w.d_v) + rows * w.d_row + rows * G * (w.d_n + w.d_v)) * e
+        step_bytes = (k_bytes + rows * w.H * w.d_v * e + w.d_row * w.hidden * e + rows * w.hidden * e
+                      + expand_bytes)
+        step_flops = k_flops + rows * 2 * w.d_row * w.hidden + rows * G * 2 * w.d_c * (w.d_n + w.d_v)
     return dict(kernel_bytes=k_bytes, kernel_flops=k_flops, step_bytes=step_bytes, step_flops=step_flops,
                 tokens=tokens)
 
@@ -252,7 +255,6 @@ def run_ours(a, rank, world, local_rank):
         G = w.n_w
         expanded = torch.empty((inp.n_pages, G, w.page, w.d_n + w.d_v), dtype=tdt, device=dev)
         mla.gqla_expand_cache(dims, W_uk, W_uv, cache, None, 0, inp.n_pages, expanded)
-        new_pages = torch.from_numpy(np.unique(inp.page_table[req_np, pos_np // w.page]).astype(np.int32)).to(dev)
         nb = mla.gqla_decode_workspace_size(dims, w.B, w.s_q, inp.seq_lens)
     else:
         nb = mla.mla_decode_workspace_size(dims, w.B, w.s_q, inp.seq_lens)
@@ -267,7 +269,8 @@ def run_ours(a, rank, world, local_rank):
         mla.mla_cache_append(dims, h, w.hidden, W_dkv, W_kr, req, pos, len(req_np), page_table, w.B, max_pages,
                              inp.n_pages, cache)
         if grouped:
-            mla.gqla_expand_cache(dims, W_uk, W_uv, cache, new_pages, len(new_pages), inp.n_pages, expanded)
+            mla.gqla_expand_tokens(dims, W_uk, W_uv, cache, req, pos, len(req_np), page_table, w.B, max_pages,
+                                   inp.n_pages, expanded)
             mla.gqla_decode_grouped(dims, q, expanded, cache, page_table, seq_lens, inp.seq_lens, w.B, w.s_q,
                                     max_pages, inp.n_pages, out, ws)
         else:

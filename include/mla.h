@@ -174,6 +174,25 @@ MLA_API mla_status gqla_expand_cache(const mla_dims *dims, const void *W_uk, con
                              const void *latent_cache, const int32_t *page_ids, int32_t n_ids,
                              int32_t n_pages_total, void *expanded_cache, mla_stream_t stream);
 
+/*
+ * gqla_expand_tokens — gqla_expand_cache for single cache rows: the rows of the tokens that
+ * mla_cache_append wrote, given by the same (req_idx, positions) arrays.  A decode step expands
+ * exactly its new tokens instead of every row of their pages.  ("GQLA ..." abstract: the GQA
+ * path's per-group expanded cache.)
+ *   req_idx, positions  device [n_tok]: request and position of each row; the row lives at
+ *                       page page_table[req_idx * max_pages + positions / page_size], row
+ *                       positions % page_size, of both caches.
+ *   page_table          device [batch, max_pages].
+ * Writes [K_g | V_g] of those rows for every group and leaves every other row untouched.
+ * Same arithmetic and rounding as gqla_expand_cache.  A row whose request, position or page id
+ * is out of range is skipped and sets MLA_ERR_DEVICE_BOUNDS; n_tok = 0 is a no-op.
+ */
+MLA_API mla_status gqla_expand_tokens(const mla_dims *dims, const void *W_uk, const void *W_uv,
+                              const void *latent_cache, const int32_t *req_idx,
+                              const int32_t *positions, int32_t n_tok, const int32_t *page_table,
+                              int32_t batch, int32_t max_pages, int32_t n_pages_total,
+                              void *expanded_cache, mla_stream_t stream);
+
 /* gqla_decode_workspace_size — as mla_decode_workspace_size, for gqla_decode_grouped. */
 MLA_API mla_status gqla_decode_workspace_size(const mla_dims *dims, int32_t batch, int32_t s_q,
                                       const int32_t *seq_lens_host, size_t *bytes);

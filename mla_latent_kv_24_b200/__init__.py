@@ -20,7 +20,7 @@ __all__ = [
     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
     "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
     "mla_decode_absorbed_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS", "mla_select_path",
-    "mla_prefill_workspace_size", "mla_prefill_expanded",
+    "mla_prefill_workspace_size", "mla_prefill_expanded", "gqla_expand_tokens",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so")
@@ -33,7 +33,7 @@ EXPORTED_SYMBOLS = ["mla_cache_append", "mla_decode_workspace_size", "mla_decode
                     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
                     "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
                     "mla_decode_absorbed_noalloc", "mla_select_path", "mla_prefill_workspace_size",
-                    "mla_prefill_expanded"]
+                    "mla_prefill_expanded", "gqla_expand_tokens"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -76,6 +76,7 @@ def load() -> ctypes.CDLL:
         "mla_decode_workspace_size": [D, _I, _I, _P, ctypes.POINTER(_S)],
         "mla_decode_absorbed": [D, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _S, _P],
         "gqla_expand_cache": [D, _P, _P, _P, _P, _I, _I, _P, _P],
+        "gqla_expand_tokens": [D, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _P, _P],
         "gqla_decode_workspace_size": [D, _I, _I, _P, ctypes.POINTER(_S)],
         "gqla_decode_grouped": [D, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _S, _P],
         "mla_get_device_status": [_P],
@@ -158,6 +159,13 @@ def gqla_expand_cache(dims, W_uk, W_uv, latent_cache, page_ids, n_ids, n_pages_t
                       stream=None) -> None:
     _check(load().gqla_expand_cache(ctypes.byref(dims), _dev(W_uk), _dev(W_uv), _dev(latent_cache), _dev(page_ids),
                                     n_ids, n_pages_total, _dev(expanded_cache), _stream(stream)))
+
+
+def gqla_expand_tokens(dims, W_uk, W_uv, latent_cache, req_idx, positions, n_tok, page_table, batch, max_pages,
+                       n_pages_total, expanded_cache, stream=None) -> None:
+    _check(load().gqla_expand_tokens(ctypes.byref(dims), _dev(W_uk), _dev(W_uv), _dev(latent_cache), _dev(req_idx),
+                                     _dev(positions), n_tok, _dev(page_table), batch, max_pages, n_pages_total,
+                                     _dev(expanded_cache), _stream(stream)))
 
 
 def gqla_decode_grouped(dims, q, expanded_cache, latent_cache, page_table, seq_lens, seq_lens_host, batch, s_q,

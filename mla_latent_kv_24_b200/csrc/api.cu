@@ -563,4 +563,27 @@ mla_status gqla_expand_cache(const mla_dims *dims, const void *W_uk, const void 
     return MLA_OK;
 }
 
+mla_status gqla_expand_tokens(const mla_dims *dims, const void *W_uk, const void *W_uv, const void *latent_cache,
+                              const int32_t *req_idx, const int32_t *positions, int32_t n_tok,
+                              const int32_t *page_table, int32_t batch, int32_t max_pages, int32_t n_pages_total,
+                              void *expanded_cache, mla_stream_t stream) {
+    g_last_error.clear();
+    Dims d;
+    MLA_TRY(check_dims(dims, &d));
+    if (n_tok < 0) return fail(MLA_ERR_INVALID_ARG, "n_tok < 0");
+    if (n_tok == 0) return MLA_OK;
+    if (!W_uk || !W_uv || !latent_cache || !expanded_cache || !req_idx || !positions || !page_table)
+        return fail(MLA_ERR_INVALID_ARG, "NULL device pointer");
+    if (batch <= 0 || max_pages <= 0 || n_pages_total <= 0)
+        return fail(MLA_ERR_INVALID_ARG, "batch, max_pages, n_pages_total must be > 0");
+    if (!aligned16(W_uk) || !aligned16(W_uv) || !aligned16(latent_cache) || !aligned16(expanded_cache))
+        return fail(MLA_ERR_INVALID_ARG, "device tensors must be 16-byte aligned");
+    int *err = nullptr;
+    MLA_TRY(device_info(&err, nullptr));
+    MLA_CUDA(launch_expand_tokens(d, W_uk, W_uv, latent_cache, req_idx, positions, n_tok, page_table, batch,
+                                  max_pages, n_pages_total, expanded_cache, err, (cudaStream_t)stream),
+             "launch gqla_expand_tokens");
+    return MLA_OK;
+}
+
 }  // extern "C"

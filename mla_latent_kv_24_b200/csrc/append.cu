@@ -117,9 +117,10 @@ cudaError_t launch_append(const Dims &d, const void *h, int hidden, const void *
 // of 256 up to 10240).  The projection [n_tok, hidden] x [hidden, 576] is weight-bandwidth bound for a
 // decode batch (n_tok = batch * s_q), so the weights must stream through many SMs at once: a
 // cluster of 8 CTAs splits the hidden dimension, each CTA multiplies its slice of 16 tokens x
-// 64 output columns with mma.sync, and rank 0 sums the 8 partial tiles through distributed
-// shared memory, then applies RoPE and scatters into the paged cache.  Grid: 9 column tiles x 8
-// hidden slices (72 CTAs) per 16-token tile.
+// 32 output columns with mma.sync (its two warp quartets taking alternate 32-wide steps of the
+// slice), and rank 0 sums the 16 partial tiles in a fixed order through distributed shared
+// memory, then applies RoPE and scatters into the paged cache.  Grid: 18 column tiles x 8 hidden
+// slices (144 CTAs, one per SM) per 16-token tile.
 // ---------------------------------------------------------------------------------------
 #include <cooperative_groups.h>
 
@@ -128,7 +129,7 @@ cudaError_t launch_append(const Dims &d, const void *h, int hidden, const void *
 namespace mla {
 namespace {
 
-constexpr int AP_SPLIT = 8, AP_COLS = 64, AP_TOK = 16;
+constexpr int AP_SPLIT = 8, AP_COLS = 32, AP_TOK = 16, AP_TILES = 576 / AP_COLS;
 
 __global__ void __cluster_dims__(AP_SPLIT, 1, 1) __launch_bounds__(256)
     append_mma_kernel(const __nv_bfloat16 *__restrict__ h, int hidden, const __nv_bfloat16 *__restrict__ W_dkv,
@@ -141,9 +142,9 @@ __global__ void __cluster_dims__(AP_SPLIT, 1, 1) __launch_bounds__(256)
     extern __shared__ __align__(16) uint8_t asm_raw[];
     const int ks = hidden / AP_SPLIT;                  // hidden slice of this CTA
     const int ld = ks + 8;
-    __nv_bfloat16 *Ws = reinterpret_cast<__nv_bfloat16 *>(asm_raw);          // [64 cols][ks]
+    __nv_bfloat16 *Ws = reinterpret_cast<__nv_bfloat16 *>(asm_raw);          // [32 cols][ks]
     __nv_bfloat16 *Hs = Ws + AP_COLS * ld;                                    // [16 tok][ks]
-    float *part = reinterpret_cast<float *>(Hs + AP_TOK * ld);                // [16][64]
+    float *part = reinterpret_cast<float *>(Hs + AP_TOK * ld);                // [2 quartets][16][32]
     const int rank = (int)cluster.block_rank();
     const int ct = blockIdx.x / AP_SPLIT, c0 = ct * AP_COLS, k0 = rank * ks;
     const int t0 = blockIdx.y * AP_TOK;
@@ -160,21 +161,24 @@ __global__ void __cluster_dims__(AP_SPLIT, 1, 1) __launch_bounds__(256)
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};   // warp w: tokens 0..15 x columns [8w, 8w + 8)
-    for (int kk = 0; kk < ks; kk += 32) {
+    // warp w: tokens 0..15 x columns [8 (w % 4), 8 (w % 4) + 8), 32-wide steps w / 4, w / 4 + 2, ...
+    const int wc = warp % 4, wq = warp / 4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int kk = 32 * wq; kk < ks; kk += 64) {
         uint32_t a0[4], a1[4], b[4];
         ldmatrix_x4(a0[0], a0[1], a0[2], a0[3], Hs + ((lane % 8) + 8 * ((lane / 8) % 2)) * ld + kk + 8 * (lane / 16));
         ldmatrix_x4(a1[0], a1[1], a1[2], a1[3],
                     Hs + ((lane % 8) + 8 * ((lane / 8) % 2)) * ld + kk + 16 + 8 * (lane / 16));
-        ldmatrix_x4(b[0], b[1], b[2], b[3], Ws + (8 * warp + (lane % 8)) * ld + kk + 8 * (lane / 8));
+        ldmatrix_x4(b[0], b[1], b[2], b[3], Ws + (8 * wc + (lane % 8)) * ld + kk + 8 * (lane / 8));
         mma_bf16(acc, a0, b[0], b[1]);
         mma_bf16(acc, a1, b[2], b[3]);
     }
     const int gid = lane / 4, t4 = lane % 4;
-    part[gid * AP_COLS + 8 * warp + 2 * t4] = acc[0];
-    part[gid * AP_COLS + 8 * warp + 2 * t4 + 1] = acc[1];
-    part[(gid + 8) * AP_COLS + 8 * warp + 2 * t4] = acc[2];
-    part[(gid + 8) * AP_COLS + 8 * warp + 2 * t4 + 1] = acc[3];
+    float *pq = part + wq * AP_TOK * AP_COLS;
+    pq[gid * AP_COLS + 8 * wc + 2 * t4] = acc[0];
+    pq[gid * AP_COLS + 8 * wc + 2 * t4 + 1] = acc[1];
+    pq[(gid + 8) * AP_COLS + 8 * wc + 2 * t4] = acc[2];
+    pq[(gid + 8) * AP_COLS + 8 * wc + 2 * t4 + 1] = acc[3];
     cluster.sync();
     if (rank == 0) {
         for (int pi = tid; pi < AP_TOK * AP_COLS / 2; pi += 256) {
@@ -185,8 +189,12 @@ __global__ void __cluster_dims__(AP_SPLIT, 1, 1) __launch_bounds__(256)
 #pragma unroll
             for (int q = 0; q < AP_SPLIT; ++q) {
                 const float *rp = cluster.map_shared_rank(part, q);
-                x0 += rp[r * AP_COLS + 2 * cp];
-                x1 += rp[r * AP_COLS + 2 * cp + 1];
+#pragma unroll
+                for (int hq = 0; hq < 2; ++hq) {
+                    const float2 x = *reinterpret_cast<const float2 *>(rp + (hq * AP_TOK + r) * AP_COLS + 2 * cp);
+                    x0 += x.x;
+                    x1 += x.y;
+                }
             }
             const int b = req[n], p = pos[n];
             if (b < 0 || b >= batch || p < 0 || p >= max_pages * 64) {
@@ -224,10 +232,10 @@ cudaError_t launch_append_mma(const Dims &d, const void *h, int hidden, const vo
                               const int *req, const int *pos, int n_tok, const int *page_table, int batch,
                               int max_pages, int n_pages, void *cache, int *err, cudaStream_t st) {
     const int ks = hidden / AP_SPLIT, ld = ks + 8;
-    const size_t smem = sizeof(__nv_bfloat16) * (size_t)(AP_COLS + AP_TOK) * ld + sizeof(float) * AP_TOK * AP_COLS;
+    const size_t smem = sizeof(__nv_bfloat16) * (size_t)(AP_COLS + AP_TOK) * ld + sizeof(float) * 2 * AP_TOK * AP_COLS;
     cudaError_t e = raise_smem_limit((const void *)append_mma_kernel, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(9 * AP_SPLIT, ceil_div(n_tok, AP_TOK));
+    dim3 grid(AP_TILES * AP_SPLIT, ceil_div(n_tok, AP_TOK));
     append_mma_kernel<<<grid, 256, smem, st>>>((const __nv_bfloat16 *)h, hidden, (const __nv_bfloat16 *)W_dkv,
                                                (const __nv_bfloat16 *)W_kr, req, pos, n_tok, page_table, batch,
                                                max_pages, n_pages, d.base, (__nv_bfloat16 *)cache, err);

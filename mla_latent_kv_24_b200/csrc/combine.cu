@@ -7,8 +7,9 @@
 // W_UV applies once to the probability-weighted latent):  out = W_UV[w(h)] O.
 // On the grouped path O already is the head's d_v-wide output.
 //
-// One CTA per (head, block of RB rows): the merged rows sit in shared memory and each W_UV
-// row is read once per RB rows.
+// Without projection, one warp merges one (row, head); with it, one CTA takes a head and a
+// block of RB rows, the merged rows sit in shared memory and each W_UV row is read once per RB
+// rows.  The bf16 DeepSeek-V2 shape takes the tensor-core kernel at the end of this file.
 #include <math.h>
 
 #include "kernels.h"
@@ -72,10 +73,82 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     }
 }
 
+// Merge without projection (grouped path, prefill): one warp per (row, head), consecutive warps
+// taking consecutive heads so a CTA reads contiguous partials; each lane owns 4 columns per
+// 128-column pass.  The chunk weights e^{m_i - M} are formed lane-parallel, the denominator
+// is summed by a fixed shuffle tree, and the partial loads are issued KB at a time.
+template <typename T>
+__global__ void __launch_bounds__(256) combine_rows_kernel(const float *__restrict__ part_o,
+                                                           const float *__restrict__ part_ml,
+                                                           const int *__restrict__ row_first, int rows, int qpi,
+                                                           int H, int DV, T *__restrict__ out) {
+    const int lane = threadIdx.x % 32;
+    const long long wid = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+    if (wid >= (long long)rows * H) return;
+    const int row = (int)(wid / H), h = (int)(wid % H);
+    const int pr = row / qpi, j = row % qpi;
+    const int k0 = row_first[pr], k1 = row_first[pr + 1];
+    auto idx = [&](int k) { return ((size_t)k * qpi + j) * H + h; };
+    float M = -INFINITY;
+    for (int k = k0 + lane; k < k1; k += 32) M = fmaxf(M, part_ml[idx(k) * 2]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float den = 0.f;
+    for (int k = k0 + lane; k < k1; k += 32) {
+        const float mk = part_ml[idx(k) * 2];
+        if (mk != -INFINITY) den += expf(mk - M) * part_ml[idx(k) * 2 + 1];
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int c = 4 * lane; c < DV; c += 128) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        constexpr int KB = 8;
+        for (int kb = k0; kb < k1; kb += KB) {
+            float4 v[KB];
+            float mk[KB];
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                mk[u] = -INFINITY;
+                if (kb + u < k1) {
+                    mk[u] = part_ml[idx(kb + u) * 2];
+                    v[u] = *reinterpret_cast<const float4 *>(part_o + idx(kb + u) * DV + c);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < KB; ++u) {
+                const float wk = mk[u] == -INFINITY ? 0.f : expf(mk[u] - M);
+                acc.x += wk * v[u].x;
+                acc.y += wk * v[u].y;
+                acc.z += wk * v[u].z;
+                acc.w += wk * v[u].w;
+            }
+        }
+        T *dst = out + ((size_t)row * H + h) * DV + c;
+        dst[0] = from_f32<T>(acc.x * inv);
+        dst[1] = from_f32<T>(acc.y * inv);
+        dst[2] = from_f32<T>(acc.z * inv);
+        dst[3] = from_f32<T>(acc.w * inv);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
                            int rows, int qpi, int DV, const void *W_uv, void *out, cudaStream_t st) {
+    if (W_uv == nullptr && DV % 4 == 0) {
+        const long long warps = (long long)rows * d.H;
+        if (warps == 0) return cudaSuccess;
+        const unsigned blocks = (unsigned)((warps + 7) / 8);
+        if (d.bf16)
+            combine_rows_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV,
+                                                                       (__nv_bfloat16 *)out);
+        else
+            combine_rows_kernel<float><<<blocks, 256, 0, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV,
+                                                               (float *)out);
+        return cudaGetLastError();
+    }
     dim3 grid(d.H, ceil_div(rows, RB));
     const size_t smem = sizeof(float) * RB * DV;
     if (d.bf16) {
@@ -97,152 +170,133 @@ cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part
 }  // namespace mla
 
 // ---------------------------------------------------------------------------------------
-// Tensor-core combine + W_UV for the DeepSeek-V2 shape (bf16, d_c = 512, d_v = 128).  One CTA
-// takes one head and 32 query rows: it merges each row's chunk partials into bf16 latent rows
-// in shared memory (the same exact merge as above), then computes out[rows, 128] =
-// O[rows, 512] W_UV[w]^T with mma.sync m16n8k16, streaming W_UV[w] in four 128-column slices
-// through a double-buffered cp.async ring.  W_UV is read once per head (16.8 MB for H = 128)
-// and the fp32 partials once.
+// Tensor-core combine + W_UV for the DeepSeek-V2 shape (bf16, d_c = 512, d_v = 128).
+//
+// A decode batch has few rows (batch x s_q) and many chunks per row, so the work of one head is
+// spread over a cluster of four CTAs, one per 128-column slice of the latent: CTA s merges the
+// chunk partials of its columns into bf16 latent rows in shared memory (the same exact merge as
+// above), multiplies them by its slice of W_UV[w] (out_s[rows, 128] = O[:, slice] W_UV[w][:, slice]^T
+// with mma.sync m16n8k16), and the four fp32 products are summed in a fixed order through
+// distributed shared memory, each CTA adding and storing 32 of the 128 output columns.  All of a
+// CTA's loads (its 32 KB of W_UV and its partials) are issued up front, and four times as many
+// SMs pull them as with one CTA per head.  W_UV is read once per head, the partials once.
 // ---------------------------------------------------------------------------------------
+#include <cooperative_groups.h>
+
 #include "warp_mma.cuh"
 
 namespace mla {
 namespace {
 
-constexpr int CM = 32, CN = 128, CK = 512, CKC = 128, O_LD = CK + 8, W_LD = CKC + 8;
+constexpr int CM = 32, CN = 128, CK = 512;                // rows per tile, d_v, d_c
+constexpr int XS = 4, XC = CK / XS, X_LD = XC + 8;        // cluster size, columns per CTA, smem row
 
 // OCT: partials in the column-octet layout [k][64][H][8] of the tcgen05 decode (else [k][H][512]).
 template <bool OCT>
-__global__ void __launch_bounds__(256) combine_mma_kernel(const float *__restrict__ part_o,
-                                                          const float *__restrict__ part_ml,
-                                                          const int *__restrict__ row_first, int rows, int H,
-                                                          const __nv_bfloat16 *__restrict__ W_uv, int hpw,
-                                                          __nv_bfloat16 *__restrict__ out) {
-    extern __shared__ __align__(16) __nv_bfloat16 csm[];
-    __nv_bfloat16 *Os = csm;                       // [64][512 + 8]
-    __nv_bfloat16 *Ws = csm + CM * O_LD;           // [2][128 v][128 + 8]
-    const int h = blockIdx.x, row0 = blockIdx.y * CM;
+__global__ void __cluster_dims__(XS, 1, 1) __launch_bounds__(256, 4)
+    combine_split_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
+                         const int *__restrict__ row_first, int rows, int H, const __nv_bfloat16 *__restrict__ W_uv,
+                         int hpw, __nv_bfloat16 *__restrict__ out) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    extern __shared__ __align__(16) uint8_t xsm[];
+    __nv_bfloat16 *Ws = reinterpret_cast<__nv_bfloat16 *>(xsm);   // [128 v][128 c + 8]
+    __nv_bfloat16 *Os = Ws + CN * X_LD;                               // [32 rows][128 c + 8]
+    float *Red = reinterpret_cast<float *>(xsm);                     // [32][128], over Ws after the MMA
+    const int s = (int)cluster.block_rank(), c0 = s * XC;
+    const int h = blockIdx.y, row0 = blockIdx.z * CM, nr = min(CM, rows - row0);
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const __nv_bfloat16 *W = W_uv + (size_t)(h / hpw) * CN * CK;
-    auto load_w = [&](int s, int c0) {
-        for (int c = tid; c < CN * CKC / 8; c += 256) {   // 2048 chunks of 16 B
-            const int v = c / (CKC / 8), k = (c % (CKC / 8)) * 8;
-            cp_async16(Ws + (s * CN + v) * W_LD + k, W + (size_t)v * CK + c0 + k, true);
-        }
-        cp_async_commit();
-    };
-    load_w(0, 0);
-    // Merge the chunk partials of every row of this tile: warp w takes rows w, w + 8, ...; lane
-    // l owns latent columns [16 l, 16 l + 16).
-    for (int r = warp; r < CM; r += 8) {
-        const int row = row0 + r;
-        float4 acc4[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (row < rows) {
+    for (int c = tid; c < CN * XC / 8; c += 256) {   // 2048 chunks of 16 B
+        const int v = c / (XC / 8), k = (c % (XC / 8)) * 8;
+        cp_async16(Ws + v * X_LD + k, W + (size_t)v * CK + c0 + k, true);
+    }
+    cp_async_commit();
+    // Merge: four rows per pass, two warps per row, each lane two adjacent columns of the slice.
+    for (int r = warp / 2; r < CM; r += 4) {
+        const int col = 64 * (warp % 2) + 2 * lane;              // column inside the slice
+        float2 acc = make_float2(0.f, 0.f);
+        if (r < nr) {
+            const int row = row0 + r;
             const int k0 = row_first[row], k1 = row_first[row + 1];
             float M = -INFINITY;
             for (int k = k0 + lane; k < k1; k += 32) M = fmaxf(M, part_ml[((size_t)k * H + h) * 2]);
 #pragma unroll
             for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
             float den = 0.f;
-            // Partials are merged in batches of KB whose loads are all issued before any is used,
-            // so a row with many chunks pays the memory latency once per batch, not per chunk.
+            // Loads are issued in batches of KB before any is used: one memory latency per batch.
             constexpr int KB = 8;
             for (int kb = k0; kb < k1; kb += KB) {
-                float4 v[KB][4];
-                float wk[KB];
+                float2 v[KB], ml[KB];
 #pragma unroll
                 for (int u = 0; u < KB; ++u) {
                     const int k = kb + u;
-                    wk[u] = 0.f;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) v[u][q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[u] = make_float2(0.f, 0.f);
+                    ml[u] = make_float2(-INFINITY, 0.f);
                     if (k < k1) {
-                        const float2 ml = *reinterpret_cast<const float2 *>(part_ml + ((size_t)k * H + h) * 2);
-                        wk[u] = ml.x == -INFINITY ? 0.f : expf(ml.x - M);
-                        den += wk[u] * ml.y;
-                        if (OCT) {
-                            const float4 *po0 = reinterpret_cast<const float4 *>(part_o + (((size_t)k * 64 + 2 * lane) * H + h) * 8);
-                            const float4 *po1 = reinterpret_cast<const float4 *>(part_o + (((size_t)k * 64 + 2 * lane + 1) * H + h) * 8);
-                            v[u][0] = po0[0];
-                            v[u][1] = po0[1];
-                            v[u][2] = po1[0];
-                            v[u][3] = po1[1];
-                        } else {
-                            const float4 *po = reinterpret_cast<const float4 *>(part_o + ((size_t)k * H + h) * CK + 16 * lane);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) v[u][q] = po[q];
-                        }
+                        ml[u] = *reinterpret_cast<const float2 *>(part_ml + ((size_t)k * H + h) * 2);
+                        const int c = c0 + col;
+                        const size_t off = OCT ? (((size_t)k * 64 + c / 8) * H + h) * 8 + c % 8
+                                               : ((size_t)k * H + h) * CK + c;
+                        v[u] = *reinterpret_cast<const float2 *>(part_o + off);
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < KB; ++u)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        acc4[q].x += wk[u] * v[u][q].x;
-                        acc4[q].y += wk[u] * v[u][q].y;
-                        acc4[q].z += wk[u] * v[u][q].z;
-                        acc4[q].w += wk[u] * v[u][q].w;
-                    }
+                for (int u = 0; u < KB; ++u) {
+                    const float wk = ml[u].x == -INFINITY ? 0.f : expf(ml[u].x - M);
+                    den += wk * ml[u].y;
+                    acc.x += wk * v[u].x;
+                    acc.y += wk * v[u].y;
+                }
             }
             const float inv = den > 0.f ? 1.f / den : 0.f;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                acc4[q].x *= inv;
-                acc4[q].y *= inv;
-                acc4[q].z *= inv;
-                acc4[q].w *= inv;
-            }
+            acc.x *= inv;
+            acc.y *= inv;
         }
-        uint4 pk0 = make_uint4(pack_bf16(acc4[0].x, acc4[0].y), pack_bf16(acc4[0].z, acc4[0].w),
-                               pack_bf16(acc4[1].x, acc4[1].y), pack_bf16(acc4[1].z, acc4[1].w));
-        uint4 pk1 = make_uint4(pack_bf16(acc4[2].x, acc4[2].y), pack_bf16(acc4[2].z, acc4[2].w),
-                               pack_bf16(acc4[3].x, acc4[3].y), pack_bf16(acc4[3].z, acc4[3].w));
-        *reinterpret_cast<uint4 *>(Os + r * O_LD + 16 * lane) = pk0;
-        *reinterpret_cast<uint4 *>(Os + r * O_LD + 16 * lane + 8) = pk1;
+        *reinterpret_cast<uint32_t *>(Os + r * X_LD + col) = pack_bf16(acc.x, acc.y);   // rows >= nr: zero
     }
+    cp_async_wait<0>();
+    __syncthreads();
     const int wm = warp % 2, wn = warp / 2;   // warp tile 16 rows x 32 columns
     float acc[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
-    for (int kc = 0; kc < CK / CKC; ++kc) {
-        if (kc + 1 < CK / CKC) {
-            load_w((kc + 1) & 1, (kc + 1) * CKC);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
-        const __nv_bfloat16 *Wt = Ws + (kc & 1) * CN * W_LD;
 #pragma unroll
-        for (int kk = 0; kk < CKC; kk += 16) {
-            uint32_t a[4];
-            ldmatrix_x4(a[0], a[1], a[2], a[3],
-                        Os + (wm * 16 + (lane % 8) + 8 * ((lane / 8) % 2)) * O_LD + kc * CKC + kk + 8 * (lane / 16));
+    for (int kk = 0; kk < XC; kk += 16) {
+        uint32_t a[4];
+        ldmatrix_x4(a[0], a[1], a[2], a[3], Os + (wm * 16 + (lane % 8) + 8 * ((lane / 8) % 2)) * X_LD + kk + 8 * (lane / 16));
 #pragma unroll
-            for (int j = 0; j < 4; j += 2) {
-                uint32_t b0, b1, b2, b3;
-                ldmatrix_x4(b0, b1, b2, b3,
-                            Wt + (wn * 32 + j * 8 + (lane % 8) + 8 * (lane / 16)) * W_LD + kk + 8 * ((lane / 8) % 2));
-                mma_bf16(acc[j], a, b0, b1);
-                mma_bf16(acc[j + 1], a, b2, b3);
-            }
+        for (int j = 0; j < 4; j += 2) {
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(b0, b1, b2, b3, Ws + (wn * 32 + j * 8 + (lane % 8) + 8 * (lane / 16)) * X_LD + kk + 8 * ((lane / 8) % 2));
+            mma_bf16(acc[j], a, b0, b1);
+            mma_bf16(acc[j + 1], a, b2, b3);
         }
-        __syncthreads();   // the next load overwrites this slice's buffer
     }
+    __syncthreads();   // Red overwrites Ws
     const int gid = lane / 4, t4 = lane % 4;
 #pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-        const int row = row0 + wm * 16 + gid + 8 * hr;
-        if (row >= rows) continue;
-        __nv_bfloat16 *dst = out + ((size_t)row * H + h) * CN + wn * 32;
+    for (int hr = 0; hr < 2; ++hr)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-            *reinterpret_cast<uint32_t *>(dst + j * 8 + 2 * t4) = pack_bf16(acc[j][2 * hr], acc[j][2 * hr + 1]);
+            *reinterpret_cast<float2 *>(Red + (wm * 16 + gid + 8 * hr) * CN + wn * 32 + j * 8 + 2 * t4) =
+                make_float2(acc[j][2 * hr], acc[j][2 * hr + 1]);
+    cluster.sync();
+    // CTA s sums output columns [32 s, 32 s + 32) over the four slices, in slice order.
+    for (int i = tid; i < nr * 16; i += 256) {
+        const int r = i / 16, v = 32 * s + 2 * (i % 16);
+        float2 sum = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < XS; ++q) {
+            const float2 x = *reinterpret_cast<const float2 *>(cluster.map_shared_rank(Red, q) + r * CN + v);
+            sum.x += x.x;
+            sum.y += x.y;
+        }
+        *reinterpret_cast<uint32_t *>(out + ((size_t)(row0 + r) * H + h) * CN + v) = pack_bf16(sum.x, sum.y);
     }
+    cluster.sync();   // the other CTAs' products stay alive until every CTA has read them
 }
 
 }  // namespace
@@ -253,9 +307,12 @@ bool combine_mma_ok(const Dims &d, int DV, bool project) {
 
 cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
                                int rows, bool oct_layout, const void *W_uv, void *out, cudaStream_t st) {
-    const size_t smem = sizeof(__nv_bfloat16) * ((size_t)CM * O_LD + 2 * (size_t)CN * W_LD);
-    dim3 grid(d.H, ceil_div(rows, CM));
-    auto k = oct_layout ? combine_mma_kernel<true> : combine_mma_kernel<false>;
+    const size_t smem = sizeof(__nv_bfloat16) * (size_t)(CN + CM) * X_LD;
+    static_assert(sizeof(float) * CM * CN <= sizeof(__nv_bfloat16) * CN * X_LD, "Red fits over Ws");
+    if (rows <= 0) return cudaSuccess;
+    if (ceil_div(rows, CM) > 65535 || d.H > 65535) return cudaErrorInvalidValue;
+    dim3 grid(XS, d.H, ceil_div(rows, CM));
+    auto k = oct_layout ? combine_split_kernel<true> : combine_split_kernel<false>;
     cudaError_t e = raise_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
     k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, d.H, (const __nv_bfloat16 *)W_uv, d.hpw,

@@ -9,6 +9,10 @@
 // slices of the latent rows and of the weight rows through a 3-stage cp.async ring into
 // padded shared memory, with mma.sync m16n8k16 and fp32 accumulators.  A CUDA-core kernel
 // covers every other shape.
+//
+// The rows to expand are either every row of a list of pages (a prefill, or a rebuild) or the
+// rows of single tokens given as (request, position) through the page table, which is how a
+// decode step expands exactly what the cache append wrote.
 #include "kernels.h"
 #include "warp_mma.cuh"
 
@@ -17,10 +21,44 @@ namespace {
 
 constexpr int BM = 128, BN = 128, BK = 64, LDS = BK + 8, STAGES = 3;
 
+// Row slot i -> (page id, row in page) of the latent / expanded caches.
+struct RowMap {
+    const int *page_ids;          // page mode: [n] page ids, or null for pages 0..n-1
+    const int *req, *pos;         // token mode (req != null): [n] request and position
+    const int *page_table;        // token mode: [batch, max_pages]
+    int n, batch, max_pages;
+    __host__ __device__ long long slots(int page) const { return req ? (long long)n : (long long)n * page; }
+};
+
+// False when slot i is past the end or names a row outside the caches (reported as a bounds error).
+__device__ __forceinline__ bool map_row(const RowMap &m, long long i, int page, int n_pages, int *pid, int *r,
+                                        int *err) {
+    if (i >= m.slots(page)) return false;
+    int p;
+    if (m.req) {
+        const int b = m.req[i], t = m.pos[i];
+        if (b < 0 || b >= m.batch || t < 0 || t >= m.max_pages * page) {
+            report(err, MLA_ERR_DEVICE_BOUNDS);
+            return false;
+        }
+        p = m.page_table[(size_t)b * m.max_pages + t / page];
+        *r = t % page;
+    } else {
+        const long long e = i / page;
+        p = m.page_ids ? m.page_ids[e] : (int)e;
+        *r = (int)(i % page);
+    }
+    if (p < 0 || p >= n_pages) {
+        report(err, MLA_ERR_DEVICE_BOUNDS);
+        return false;
+    }
+    *pid = p;
+    return true;
+}
+
 __global__ void __launch_bounds__(256) expand_mma_kernel(const __nv_bfloat16 *__restrict__ W_uk,
                                                          const __nv_bfloat16 *__restrict__ W_uv,
-                                                         const __nv_bfloat16 *__restrict__ latent,
-                                                         const int *__restrict__ page_ids, int n_ids,
+                                                         const __nv_bfloat16 *__restrict__ latent, RowMap map,
                                                          int n_pages, int page, int d_c, int d_r, int G,
                                                          __nv_bfloat16 *__restrict__ out, int *err) {
     extern __shared__ __align__(16) __nv_bfloat16 sm[];
@@ -35,17 +73,11 @@ __global__ void __launch_bounds__(256) expand_mma_kernel(const __nv_bfloat16 *__
     const __nv_bfloat16 *W = (half == 0 ? W_uk : W_uv) + (size_t)g * 128 * d_c;
 
     if (tid < BM) {
-        const long long i = (long long)blockIdx.x * BM + tid;
-        const long long e = i / page, r = i % page;
+        int pid, r;
         long long ro = -1, oo = -1;
-        if (e < n_ids) {
-            const int pid = page_ids ? page_ids[e] : (int)e;
-            if (pid < 0 || pid >= n_pages) {
-                report(err, MLA_ERR_DEVICE_BOUNDS);
-            } else {
-                ro = ((long long)pid * page + r) * d_row;
-                oo = (((long long)pid * G + g) * page + r) * 256 + half * 128;
-            }
+        if (map_row(map, (long long)blockIdx.x * BM + tid, page, n_pages, &pid, &r, err)) {
+            ro = ((long long)pid * page + r) * d_row;
+            oo = (((long long)pid * G + g) * page + r) * 256 + half * 128;
         }
         row_off[tid] = ro;
         out_off[tid] = oo;
@@ -128,24 +160,17 @@ __global__ void __launch_bounds__(256) expand_mma_kernel(const __nv_bfloat16 *__
 // CUDA-core expansion for other shapes / fp32: one thread per output element.
 template <typename T>
 __global__ void expand_simt_kernel(const T *__restrict__ W_uk, const T *__restrict__ W_uv,
-                                   const T *__restrict__ latent, const int *__restrict__ page_ids, int n_ids,
-                                   int n_pages, int page, int d_c, int d_r, int d_n, int d_v, int G,
-                                   T *__restrict__ out, int *err) {
+                                   const T *__restrict__ latent, RowMap map, int n_pages, int page, int d_c,
+                                   int d_r, int d_n, int d_v, int G, T *__restrict__ out, int *err) {
     const int w_out = d_n + d_v;
-    const long long n = (long long)n_ids * page * G * w_out;
+    const long long n = map.slots(page) * G * w_out;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
          i += (long long)gridDim.x * blockDim.x) {
         const int o = (int)(i % w_out);
-        long long rest = i / w_out;
+        const long long rest = i / w_out;
         const int g = (int)(rest % G);
-        rest /= G;
-        const int r = (int)(rest % page);
-        const long long e = rest / page;
-        const int pid = page_ids ? page_ids[e] : (int)e;
-        if (pid < 0 || pid >= n_pages) {
-            report(err, MLA_ERR_DEVICE_BOUNDS);
-            continue;
-        }
+        int pid, r;
+        if (!map_row(map, rest / G, page, n_pages, &pid, &r, err)) continue;
         const T *c = latent + ((size_t)pid * page + r) * (d_c + d_r);
         const T *w = o < d_n ? W_uk + ((size_t)g * d_n + o) * d_c : W_uv + ((size_t)g * d_v + (o - d_n)) * d_c;
         float acc = 0.f;
@@ -156,32 +181,46 @@ __global__ void expand_simt_kernel(const T *__restrict__ W_uk, const T *__restri
 
 }  // namespace
 
-cudaError_t launch_expand(const Dims &d, const void *W_uk, const void *W_uv, const void *latent,
-                          const int *page_ids, int n_ids, int n_pages, void *expanded, int *err,
-                          cudaStream_t st) {
+static cudaError_t launch_expand_rows(const Dims &d, const void *W_uk, const void *W_uv, const void *latent,
+                                      const RowMap &map, int n_pages, void *expanded, int *err, cudaStream_t st) {
     const int G = d.n_groups();
-    if (n_ids == 0) return cudaSuccess;
+    const long long slots = map.slots(d.page);
+    if (slots == 0) return cudaSuccess;
     if (d.bf16 && d.d_n == 128 && d.d_v == 128 && d.d_c % BK == 0) {
         const size_t smem = sizeof(__nv_bfloat16) * STAGES * (BM + BN) * LDS;
         cudaError_t e = raise_smem_limit((const void *)expand_mma_kernel, smem);
         if (e != cudaSuccess) return e;
-        dim3 grid((unsigned)(((long long)n_ids * d.page + BM - 1) / BM), G, 2);
+        dim3 grid((unsigned)((slots + BM - 1) / BM), G, 2);
         expand_mma_kernel<<<grid, 256, smem, st>>>((const __nv_bfloat16 *)W_uk, (const __nv_bfloat16 *)W_uv,
-                                                   (const __nv_bfloat16 *)latent, page_ids, n_ids, n_pages, d.page,
-                                                   d.d_c, d.d_r, G, (__nv_bfloat16 *)expanded, err);
+                                                   (const __nv_bfloat16 *)latent, map, n_pages, d.page, d.d_c, d.d_r,
+                                                   G, (__nv_bfloat16 *)expanded, err);
         return cudaGetLastError();
     }
-    const long long n = (long long)n_ids * d.page * G * (d.d_n + d.d_v);
+    const long long n = slots * G * (d.d_n + d.d_v);
     const int blocks = (int)std::min<long long>((n + 255) / 256, 65535);
     if (d.bf16)
         expand_simt_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-            (const __nv_bfloat16 *)W_uk, (const __nv_bfloat16 *)W_uv, (const __nv_bfloat16 *)latent, page_ids, n_ids,
-            n_pages, d.page, d.d_c, d.d_r, d.d_n, d.d_v, G, (__nv_bfloat16 *)expanded, err);
+            (const __nv_bfloat16 *)W_uk, (const __nv_bfloat16 *)W_uv, (const __nv_bfloat16 *)latent, map, n_pages,
+            d.page, d.d_c, d.d_r, d.d_n, d.d_v, G, (__nv_bfloat16 *)expanded, err);
     else
         expand_simt_kernel<float><<<blocks, 256, 0, st>>>((const float *)W_uk, (const float *)W_uv,
-                                                          (const float *)latent, page_ids, n_ids, n_pages, d.page,
-                                                          d.d_c, d.d_r, d.d_n, d.d_v, G, (float *)expanded, err);
+                                                          (const float *)latent, map, n_pages, d.page, d.d_c, d.d_r,
+                                                          d.d_n, d.d_v, G, (float *)expanded, err);
     return cudaGetLastError();
+}
+
+cudaError_t launch_expand(const Dims &d, const void *W_uk, const void *W_uv, const void *latent,
+                          const int *page_ids, int n_ids, int n_pages, void *expanded, int *err,
+                          cudaStream_t st) {
+    const RowMap map{page_ids, nullptr, nullptr, nullptr, n_ids, 0, 0};
+    return launch_expand_rows(d, W_uk, W_uv, latent, map, n_pages, expanded, err, st);
+}
+
+cudaError_t launch_expand_tokens(const Dims &d, const void *W_uk, const void *W_uv, const void *latent,
+                                 const int *req, const int *pos, int n_tok, const int *page_table, int batch,
+                                 int max_pages, int n_pages, void *expanded, int *err, cudaStream_t st) {
+    const RowMap map{nullptr, req, pos, page_table, n_tok, batch, max_pages};
+    return launch_expand_rows(d, W_uk, W_uv, latent, map, n_pages, expanded, err, st);
 }
 
 }  // namespace mla

@@ -81,5 +81,8 @@ cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *
 cudaError_t launch_expand(const Dims &d, const void *W_uk, const void *W_uv, const void *latent,
                           const int *page_ids, int n_ids, int n_pages, void *expanded, int *err,
                           cudaStream_t st);
+cudaError_t launch_expand_tokens(const Dims &d, const void *W_uk, const void *W_uv, const void *latent,
+                                 const int *req, const int *pos, int n_tok, const int *page_table, int batch,
+                                 int max_pages, int n_pages, void *expanded, int *err, cudaStream_t st);
 
 }  // namespace mla

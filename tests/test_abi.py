@@ -85,3 +85,15 @@ def test_prefill_argument_checks_without_device():
     a = mla.mla_prefill_workspace_size(dims, 2, 16, [100, 500])
     b = mla.mla_prefill_workspace_size(dims, 2, 32, [100, 500])
     assert 1.9 < b / a < 2.1
+
+
+def test_expand_tokens_argument_checks():
+    lib = mla.load()
+    d = mla.make_dims()
+    # zero tokens is a no-op, whatever the pointers
+    assert lib.gqla_expand_tokens(ctypes.byref(d), None, None, None, None, None, 0, None, 1, 1, 1, None, None) == 0
+    assert lib.gqla_expand_tokens(ctypes.byref(d), 256, 256, 256, 256, 256, -1, 256, 1, 1, 1, 256, None) == 1
+    assert lib.gqla_expand_tokens(ctypes.byref(d), 256, 256, 256, None, 256, 4, 256, 1, 1, 1, 256, None) == 1
+    assert lib.gqla_expand_tokens(ctypes.byref(d), 256, 256, 256, 256, 256, 4, 256, 0, 1, 1, 256, None) == 1
+    assert lib.gqla_expand_tokens(ctypes.byref(d), 256, 256, 8, 256, 256, 4, 256, 1, 1, 1, 256, None) == 1
+    assert "aligned" in mla.mla_last_error_string()
