@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(256) q_absorb_kernel(const T *__restrict__ q, 
                                                        const int *__restrict__ seq_lens, int rows, int s_q,
                                                        int H, int hpw, int d_c, int d_r, int d_n, float base,
                                                        T *__restrict__ q_abs) {
+    step_begin();
     __shared__ float qn[RB][128];
     const int h = blockIdx.x, w = h / hpw;
     const int row0 = blockIdx.y * RB;
@@ -61,6 +62,7 @@ __global__ void __launch_bounds__(256) q_absorb_kernel(const T *__restrict__ q, 
 template <typename T>
 __global__ void q_rope_kernel(const T *__restrict__ q, const int *__restrict__ seq_lens, int rows, int s_q,
                               int H, int d_r, int d_n, float base, T *__restrict__ q_rot) {
+    step_begin();
     const int d_qk = d_n + d_r;
     const size_t n = (size_t)rows * H * (d_qk / 2);
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
@@ -89,12 +91,12 @@ cudaError_t launch_q_absorb(const Dims &d, const void *q, const void *W_uk, cons
     const int rows = batch * s_q;
     dim3 grid(d.H, ceil_div(rows, RB));
     if (d.bf16)
-        q_absorb_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-            (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)W_uk, seq_lens, rows, s_q, d.H, d.hpw, d.d_c,
-            d.d_r, d.d_n, d.base, (__nv_bfloat16 *)q_abs);
+        MLA_STEP_LAUNCH(q_absorb_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, (const __nv_bfloat16 *)q,
+                        (const __nv_bfloat16 *)W_uk, seq_lens, rows, s_q, d.H, d.hpw, d.d_c, d.d_r, d.d_n, d.base,
+                        (__nv_bfloat16 *)q_abs);
     else
-        q_absorb_kernel<float><<<grid, 256, 0, st>>>((const float *)q, (const float *)W_uk, seq_lens, rows, s_q,
-                                                     d.H, d.hpw, d.d_c, d.d_r, d.d_n, d.base, (float *)q_abs);
+        MLA_STEP_LAUNCH(q_absorb_kernel<float>, dim3(grid), dim3(256), 0, st, (const float *)q, (const float *)W_uk,
+                        seq_lens, rows, s_q, d.H, d.hpw, d.d_c, d.d_r, d.d_n, d.base, (float *)q_abs);
     return cudaGetLastError();
 }
 
@@ -104,11 +106,11 @@ cudaError_t launch_q_rope(const Dims &d, const void *q, const int *seq_lens, int
     const size_t n = (size_t)rows * d.H * ((d.d_n + d.d_r) / 2);
     const int blocks = (int)std::min<size_t>((n + 255) / 256, 4096);
     if (d.bf16)
-        q_rope_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)q, seq_lens, rows, s_q, d.H,
-                                                              d.d_r, d.d_n, d.base, (__nv_bfloat16 *)q_rot);
+        MLA_STEP_LAUNCH(q_rope_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, (const __nv_bfloat16 *)q,
+                        seq_lens, rows, s_q, d.H, d.d_r, d.d_n, d.base, (__nv_bfloat16 *)q_rot);
     else
-        q_rope_kernel<float><<<blocks, 256, 0, st>>>((const float *)q, seq_lens, rows, s_q, d.H, d.d_r, d.d_n,
-                                                     d.base, (float *)q_rot);
+        MLA_STEP_LAUNCH(q_rope_kernel<float>, dim3(blocks), dim3(256), 0, st, (const float *)q, seq_lens, rows, s_q,
+                        d.H, d.d_r, d.d_n, d.base, (float *)q_rot);
     return cudaGetLastError();
 }
 
@@ -135,6 +137,7 @@ __global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *
                                                            const int *__restrict__ seq_lens, int rows, int s_q,
                                                            int H, int hpw, float base,
                                                            __nv_bfloat16 *__restrict__ q_abs) {
+    step_begin();
     __shared__ __align__(16) __nv_bfloat16 As[AB_M * AB_LD];    // [64 rows][128 k]
     __shared__ __align__(16) __nv_bfloat16 Bs[AB_K * AB_LDB];   // [128 k][64 n]
     const int h = blockIdx.x, n0 = blockIdx.y * AB_N, row0 = blockIdx.z * AB_M;
@@ -209,8 +212,8 @@ cudaError_t launch_q_absorb_mma(const Dims &d, const void *q, const void *W_uk, 
                                 int s_q, void *q_abs, cudaStream_t st) {
     const int rows = batch * s_q;
     dim3 grid(d.H, 512 / AB_N, ceil_div(rows, AB_M));
-    q_absorb_mma_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16 *)q, (const __nv_bfloat16 *)W_uk, seq_lens, rows,
-                                              s_q, d.H, d.hpw, d.base, (__nv_bfloat16 *)q_abs);
+    MLA_STEP_LAUNCH(q_absorb_mma_kernel, dim3(grid), dim3(256), 0, st, (const __nv_bfloat16 *)q,
+                    (const __nv_bfloat16 *)W_uk, seq_lens, rows, s_q, d.H, d.hpw, d.base, (__nv_bfloat16 *)q_abs);
     return cudaGetLastError();
 }
 

@@ -20,6 +20,7 @@ __global__ void __launch_bounds__(256) append_kernel(
     const int *__restrict__ req, const int *__restrict__ pos, int n_tok,
     const int *__restrict__ page_table, int batch, int max_pages, int n_pages, int page, int d_c,
     int d_r, float base, T *__restrict__ cache, int *err) {
+    step_begin();
     const int d_row = d_c + d_r;
     __shared__ float hs[TOK][KT + 1];
     __shared__ float ws[COLS][KT + 1];
@@ -99,14 +100,13 @@ cudaError_t launch_append(const Dims &d, const void *h, int hidden, const void *
                           void *cache, int *err, cudaStream_t st) {
     dim3 grid(ceil_div(d.d_row(), COLS), ceil_div(n_tok, TOK));
     if (d.bf16)
-        append_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-            (const __nv_bfloat16 *)h, hidden, (const __nv_bfloat16 *)W_dkv, (const __nv_bfloat16 *)W_kr,
-            req, pos, n_tok, page_table, batch, max_pages, n_pages, d.page, d.d_c, d.d_r, d.base,
-            (__nv_bfloat16 *)cache, err);
+        MLA_STEP_LAUNCH(append_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, (const __nv_bfloat16 *)h, hidden,
+                        (const __nv_bfloat16 *)W_dkv, (const __nv_bfloat16 *)W_kr, req, pos, n_tok, page_table, batch,
+                        max_pages, n_pages, d.page, d.d_c, d.d_r, d.base, (__nv_bfloat16 *)cache, err);
     else
-        append_kernel<float><<<grid, 256, 0, st>>>(
-            (const float *)h, hidden, (const float *)W_dkv, (const float *)W_kr, req, pos, n_tok,
-            page_table, batch, max_pages, n_pages, d.page, d.d_c, d.d_r, d.base, (float *)cache, err);
+        MLA_STEP_LAUNCH(append_kernel<float>, dim3(grid), dim3(256), 0, st, (const float *)h, hidden,
+                        (const float *)W_dkv, (const float *)W_kr, req, pos, n_tok, page_table, batch, max_pages,
+                        n_pages, d.page, d.d_c, d.d_r, d.base, (float *)cache, err);
     return cudaGetLastError();
 }
 
@@ -136,6 +136,7 @@ __global__ void __cluster_dims__(AP_SPLIT, 1, 1) __launch_bounds__(256)
                       const __nv_bfloat16 *__restrict__ W_kr, const int *__restrict__ req,
                       const int *__restrict__ pos, int n_tok, const int *__restrict__ page_table, int batch,
                       int max_pages, int n_pages, float base, __nv_bfloat16 *__restrict__ cache, int *err) {
+    step_begin();
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     constexpr int D_C = 512, D_R = 64, D_ROW = 576;
@@ -236,9 +237,9 @@ cudaError_t launch_append_mma(const Dims &d, const void *h, int hidden, const vo
     cudaError_t e = raise_smem_limit((const void *)append_mma_kernel, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(AP_TILES * AP_SPLIT, ceil_div(n_tok, AP_TOK));
-    append_mma_kernel<<<grid, 256, smem, st>>>((const __nv_bfloat16 *)h, hidden, (const __nv_bfloat16 *)W_dkv,
-                                               (const __nv_bfloat16 *)W_kr, req, pos, n_tok, page_table, batch,
-                                               max_pages, n_pages, d.base, (__nv_bfloat16 *)cache, err);
+    MLA_STEP_LAUNCH(append_mma_kernel, dim3(grid), dim3(256), smem, st, (const __nv_bfloat16 *)h, hidden,
+                    (const __nv_bfloat16 *)W_dkv, (const __nv_bfloat16 *)W_kr, req, pos, n_tok, page_table, batch,
+                    max_pages, n_pages, d.base, (__nv_bfloat16 *)cache, err);
     return cudaGetLastError();
 }
 

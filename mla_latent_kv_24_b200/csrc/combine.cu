@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
                                                       const int *__restrict__ row_first, int rows, int qpi,
                                                       int H, int DV, const T *__restrict__ W_uv, int hpw,
                                                       int d_v, T *__restrict__ out) {
+    step_begin();
     extern __shared__ float O[];  // [RB][DV]
     const int h = blockIdx.x;
     const int row0 = blockIdx.y * RB;
@@ -82,6 +83,7 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(const float *__restri
                                                            const float *__restrict__ part_ml,
                                                            const int *__restrict__ row_first, int rows, int qpi,
                                                            int H, int DV, T *__restrict__ out) {
+    step_begin();
     const int lane = threadIdx.x % 32;
     const long long wid = (long long)blockIdx.x * 8 + threadIdx.x / 32;
     if (wid >= (long long)rows * H) return;
@@ -142,11 +144,11 @@ cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part
         if (warps == 0) return cudaSuccess;
         const unsigned blocks = (unsigned)((warps + 7) / 8);
         if (d.bf16)
-            combine_rows_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV,
-                                                                       (__nv_bfloat16 *)out);
+            MLA_STEP_LAUNCH(combine_rows_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, part_o, part_ml,
+                            row_first, rows, qpi, d.H, DV, (__nv_bfloat16 *)out);
         else
-            combine_rows_kernel<float><<<blocks, 256, 0, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV,
-                                                               (float *)out);
+            MLA_STEP_LAUNCH(combine_rows_kernel<float>, dim3(blocks), dim3(256), 0, st, part_o, part_ml, row_first,
+                            rows, qpi, d.H, DV, (float *)out);
         return cudaGetLastError();
     }
     dim3 grid(d.H, ceil_div(rows, RB));
@@ -155,14 +157,14 @@ cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part
         auto k = combine_kernel<__nv_bfloat16>;
         cudaError_t e = raise_smem_limit((const void *)k, smem);
         if (e != cudaSuccess) return e;
-        k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV, (const __nv_bfloat16 *)W_uv,
-                                   d.hpw, d.d_v, (__nv_bfloat16 *)out);
+        MLA_STEP_LAUNCH(k, dim3(grid), dim3(256), smem, st, part_o, part_ml, row_first, rows, qpi, d.H, DV,
+                        (const __nv_bfloat16 *)W_uv, d.hpw, d.d_v, (__nv_bfloat16 *)out);
     } else {
         auto k = combine_kernel<float>;
         cudaError_t e = raise_smem_limit((const void *)k, smem);
         if (e != cudaSuccess) return e;
-        k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, qpi, d.H, DV, (const float *)W_uv, d.hpw, d.d_v,
-                                   (float *)out);
+        MLA_STEP_LAUNCH(k, dim3(grid), dim3(256), smem, st, part_o, part_ml, row_first, rows, qpi, d.H, DV,
+                        (const float *)W_uv, d.hpw, d.d_v, (float *)out);
     }
     return cudaGetLastError();
 }
@@ -197,6 +199,7 @@ __global__ void __cluster_dims__(XS, 1, 1) __launch_bounds__(256, 4)
     combine_split_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
                          const int *__restrict__ row_first, int rows, int H, const __nv_bfloat16 *__restrict__ W_uv,
                          int hpw, __nv_bfloat16 *__restrict__ out) {
+    step_begin();
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     extern __shared__ __align__(16) uint8_t xsm[];
@@ -315,8 +318,8 @@ cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *
     auto k = oct_layout ? combine_split_kernel<true> : combine_split_kernel<false>;
     cudaError_t e = raise_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, 256, smem, st>>>(part_o, part_ml, row_first, rows, d.H, (const __nv_bfloat16 *)W_uv, d.hpw,
-                               (__nv_bfloat16 *)out);
+    MLA_STEP_LAUNCH(k, dim3(grid), dim3(256), smem, st, part_o, part_ml, row_first, rows, d.H,
+                    (const __nv_bfloat16 *)W_uv, d.hpw, (__nv_bfloat16 *)out);
     return cudaGetLastError();
 }
 

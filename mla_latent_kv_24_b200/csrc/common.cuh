@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <utility>
 
 #include "mla.h"
 
@@ -46,6 +47,21 @@ __device__ __forceinline__ void rope_cos_sin(int pos, int i, int d, float base, 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // ---------------------------------------------------------------------------------------
+// Programmatic dependent launch.  The kernels of a call are launched with programmatic stream
+// serialisation, so a kernel's CTAs may be launched while the previous kernel of the stream is
+// still running.  Every such kernel calls step_begin() before anything else: it waits until the
+// previous kernel has completed and its writes are visible (griddepcontrol.wait), then allows
+// the next kernel to start launching (griddepcontrol.launch_dependents).  Execution order and
+// memory order therefore stay those of a plain stream, and only the launch latency of the next
+// kernel overlaps this one.  Both instructions do nothing in a kernel launched without the
+// attribute.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void step_begin() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------------
 // Split-KV plan.  Row r = (b, j) has len_r = seq_lens[b] - s_q + j + 1 visible tokens and
 // is cut into ceil(len_r / chunk) chunks of `chunk` tokens (the last one ragged).  Work item
 // k covers tokens [t0, t1) of one row; partial results are stored at index k.
@@ -67,6 +83,31 @@ struct Plan {
 }  // namespace mla
 
 namespace mla {
+// Launches `kernel` on `st` with programmatic stream serialisation (the kernel must call
+// step_begin() first).  Host only.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_step(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                               Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// One statement: launch with launch_step() and return its error, if any, from the caller.
+#define MLA_STEP_LAUNCH(kernel, grid, block, smem, st, ...)                                       \
+    do {                                                                                          \
+        const cudaError_t e_launch_ = ::mla::launch_step(kernel, grid, block, smem, st, __VA_ARGS__); \
+        if (e_launch_ != cudaSuccess) return e_launch_;                                           \
+    } while (0)
+
 // Raises a kernel's dynamic shared-memory limit on the current device once, to the largest size
 // asked so far; later launches that need no more skip the driver call (it costs microseconds of
 // host time per launch).  Host only; thread-safe.

@@ -56,6 +56,7 @@ struct GParams {
 // Prefill: CTA = (head, item, query tile), row m = query 16 * tile + m of that head.
 template <bool PREFILL>
 __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p) {
+    step_begin();
     extern __shared__ __align__(16) uint8_t gsm[];
     __nv_bfloat16 *kv = reinterpret_cast<__nv_bfloat16 *>(gsm);           // [STAGES][64][KV_LD]
     __nv_bfloat16 *kr = kv + STAGES * KV_TILE;                            // [STAGES][64][KR_LD]
@@ -314,7 +315,7 @@ cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expa
     cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<false>, SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(d.H / GH, std::min(plan.n_work, 65535), ceil_div(plan.n_work, 65535));
-    grouped_decode_kernel<false><<<grid, WARPS * 32, SMEM, st>>>(p);
+    MLA_STEP_LAUNCH(grouped_decode_kernel<false>, dim3(grid), dim3(WARPS * 32), SMEM, st, p);
     return cudaGetLastError();
 }
 
@@ -332,7 +333,7 @@ cudaError_t launch_prefill_expanded(const Dims &d, const void *q_rot, const void
     cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<true>, SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(d.H, plan.n_work, ceil_div(n_q, 16));
-    grouped_decode_kernel<true><<<grid, WARPS * 32, SMEM, st>>>(p);
+    MLA_STEP_LAUNCH(grouped_decode_kernel<true>, dim3(grid), dim3(WARPS * 32), SMEM, st, p);
     return cudaGetLastError();
 }
 

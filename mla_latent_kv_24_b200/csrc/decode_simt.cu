@@ -45,6 +45,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 template <typename T, int MODE>
 __global__ void __launch_bounds__(WARPS * 32) decode_simt_kernel(P p) {
+    step_begin();
     extern __shared__ float smem[];
     const int KS = p.DK + 1, VS = p.DV + 1;
     float *qs = smem;                         // [HB][DK]
@@ -174,7 +175,7 @@ cudaError_t launch_t(const P &p, dim3 grid, size_t smem, cudaStream_t st) {
     auto k = decode_simt_kernel<T, MODE>;
     cudaError_t e = raise_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
-    k<<<grid, WARPS * 32, smem, st>>>(p);
+    MLA_STEP_LAUNCH(k, dim3(grid), dim3(WARPS * 32), smem, st, p);
     return cudaGetLastError();
 }
 

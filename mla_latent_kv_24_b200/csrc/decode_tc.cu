@@ -416,6 +416,7 @@ __device__ void run_softmax(const Ctx &c, const TcParams &p, uint32_t tmem, int 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, TcParams p) {
+    step_begin();
     extern __shared__ uint8_t smem_raw[];
     Ctx c;
     const uint32_t raw = tc::smem_addr(smem_raw);
@@ -594,7 +595,7 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
     cudaError_t e = raise_smem_limit((const void *)tc_decode_kernel, SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     const int units = std::max(1, std::min(plan.n_work, std::max(1, sms / 2)));
-    tc_decode_kernel<<<2 * units, THREADS, SMEM_ALLOC, st>>>(tm_q, tm_k, tm_v, p);
+    MLA_STEP_LAUNCH(tc_decode_kernel, dim3(2 * units), dim3(THREADS), SMEM_ALLOC, st, tm_q, tm_k, tm_v, p);
     return cudaGetLastError();
 }
 

@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(256) expand_mma_kernel(const __nv_bfloat16 *__
                                                          const __nv_bfloat16 *__restrict__ latent, RowMap map,
                                                          int n_pages, int page, int d_c, int d_r, int G,
                                                          __nv_bfloat16 *__restrict__ out, int *err) {
+    step_begin();
     extern __shared__ __align__(16) __nv_bfloat16 sm[];
     __nv_bfloat16 *As = sm;                          // [STAGES][BM][LDS]
     __nv_bfloat16 *Bs = sm + STAGES * BM * LDS;      // [STAGES][BN][LDS]
@@ -162,6 +163,7 @@ template <typename T>
 __global__ void expand_simt_kernel(const T *__restrict__ W_uk, const T *__restrict__ W_uv,
                                    const T *__restrict__ latent, RowMap map, int n_pages, int page, int d_c,
                                    int d_r, int d_n, int d_v, int G, T *__restrict__ out, int *err) {
+    step_begin();
     const int w_out = d_n + d_v;
     const long long n = map.slots(page) * G * w_out;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
@@ -191,21 +193,21 @@ static cudaError_t launch_expand_rows(const Dims &d, const void *W_uk, const voi
         cudaError_t e = raise_smem_limit((const void *)expand_mma_kernel, smem);
         if (e != cudaSuccess) return e;
         dim3 grid((unsigned)((slots + BM - 1) / BM), G, 2);
-        expand_mma_kernel<<<grid, 256, smem, st>>>((const __nv_bfloat16 *)W_uk, (const __nv_bfloat16 *)W_uv,
-                                                   (const __nv_bfloat16 *)latent, map, n_pages, d.page, d.d_c, d.d_r,
-                                                   G, (__nv_bfloat16 *)expanded, err);
+        MLA_STEP_LAUNCH(expand_mma_kernel, dim3(grid), dim3(256), smem, st, (const __nv_bfloat16 *)W_uk,
+                        (const __nv_bfloat16 *)W_uv, (const __nv_bfloat16 *)latent, map, n_pages, d.page, d.d_c,
+                        d.d_r, G, (__nv_bfloat16 *)expanded, err);
         return cudaGetLastError();
     }
     const long long n = slots * G * (d.d_n + d.d_v);
     const int blocks = (int)std::min<long long>((n + 255) / 256, 65535);
     if (d.bf16)
-        expand_simt_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-            (const __nv_bfloat16 *)W_uk, (const __nv_bfloat16 *)W_uv, (const __nv_bfloat16 *)latent, map, n_pages,
-            d.page, d.d_c, d.d_r, d.d_n, d.d_v, G, (__nv_bfloat16 *)expanded, err);
+        MLA_STEP_LAUNCH(expand_simt_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
+                        (const __nv_bfloat16 *)W_uk, (const __nv_bfloat16 *)W_uv, (const __nv_bfloat16 *)latent, map,
+                        n_pages, d.page, d.d_c, d.d_r, d.d_n, d.d_v, G, (__nv_bfloat16 *)expanded, err);
     else
-        expand_simt_kernel<float><<<blocks, 256, 0, st>>>((const float *)W_uk, (const float *)W_uv,
-                                                          (const float *)latent, map, n_pages, d.page, d.d_c, d.d_r,
-                                                          d.d_n, d.d_v, G, (float *)expanded, err);
+        MLA_STEP_LAUNCH(expand_simt_kernel<float>, dim3(blocks), dim3(256), 0, st, (const float *)W_uk,
+                        (const float *)W_uv, (const float *)latent, map, n_pages, d.page, d.d_c, d.d_r, d.d_n, d.d_v,
+                        G, (float *)expanded, err);
     return cudaGetLastError();
 }
 

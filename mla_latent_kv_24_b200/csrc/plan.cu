@@ -15,6 +15,7 @@ __global__ void __launch_bounds__(PT) plan_kernel(const int *__restrict__ seq_le
                                                   int max_pages, int page, int chunk, int n_expected,
                                                   WorkItem *__restrict__ items, int *__restrict__ row_first,
                                                   int *err) {
+    step_begin();
     __shared__ int warp_sum[PT / 32];
     __shared__ int bad;
     const int rows = batch * s_q;
@@ -86,8 +87,8 @@ __global__ void __launch_bounds__(PT) plan_kernel(const int *__restrict__ seq_le
 
 cudaError_t launch_plan(const int *seq_lens, int batch, int s_q, int max_pages, int page, int chunk,
                         int n_work_expected, WorkItem *items, int *row_first, int *err, cudaStream_t st) {
-    plan_kernel<<<1, PT, 0, st>>>(seq_lens, batch, s_q, max_pages, page, chunk, n_work_expected, items,
-                                  row_first, err);
+    MLA_STEP_LAUNCH(plan_kernel, dim3(1), dim3(PT), 0, st, seq_lens, batch, s_q, max_pages, page, chunk,
+                    n_work_expected, items, row_first, err);
     return cudaGetLastError();
 }
 
