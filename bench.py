@@ -352,7 +352,7 @@ def run_ours(a, rank, world, local_rank):
         achieved = kb / ks / 1e9 if bound == "hbm" else kf / ks / 1e12
         peak = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"]
         traffic = recorded_traffic(a.path, a.workload)
-        launches_per_step = 6 if grouped else 5   # append, (expand,) plan, q absorb or q RoPE, decode, combine
+        launches_per_step = 5 if grouped else 4   # append, (expand,) q absorb or q RoPE with the plan, decode, combine
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

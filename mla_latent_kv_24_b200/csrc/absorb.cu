@@ -10,6 +10,7 @@
 // One CTA handles one head and up to RB query rows, so each W_UK row is read once per RB
 // rows; every thread owns two latent columns.
 #include "kernels.h"
+#include "plan_block.cuh"
 
 namespace mla {
 namespace {
@@ -59,13 +60,20 @@ __global__ void __launch_bounds__(256) q_absorb_kernel(const T *__restrict__ q, 
 }
 
 // GQA path: the no-position part is used as is; only the RoPE part turns.
+// The last block builds the split plan instead.
 template <typename T>
-__global__ void q_rope_kernel(const T *__restrict__ q, const int *__restrict__ seq_lens, int rows, int s_q,
-                              int H, int d_r, int d_n, float base, T *__restrict__ q_rot) {
+__global__ void __launch_bounds__(256) q_rope_kernel(const T *__restrict__ q, const int *__restrict__ seq_lens,
+                                                     int rows, int s_q, int H, int d_r, int d_n, float base,
+                                                     T *__restrict__ q_rot, PlanArgs plan) {
     step_begin();
+    if (blockIdx.x == gridDim.x - 1) {
+        plan_block<256>(plan);
+        return;
+    }
     const int d_qk = d_n + d_r;
     const size_t n = (size_t)rows * H * (d_qk / 2);
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t stride = (size_t)(gridDim.x - 1) * blockDim.x;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += stride) {
         const int pr = (int)(i % (d_qk / 2));
         const size_t rh = i / (d_qk / 2);
         const int row = (int)(rh / H);
@@ -101,16 +109,16 @@ cudaError_t launch_q_absorb(const Dims &d, const void *q, const void *W_uk, cons
 }
 
 cudaError_t launch_q_rope(const Dims &d, const void *q, const int *seq_lens, int batch, int s_q, void *q_rot,
-                          cudaStream_t st) {
+                          const PlanArgs &plan, cudaStream_t st) {
     const int rows = batch * s_q;
     const size_t n = (size_t)rows * d.H * ((d.d_n + d.d_r) / 2);
-    const int blocks = (int)std::min<size_t>((n + 255) / 256, 4096);
+    const int blocks = (int)std::min<size_t>((n + 255) / 256, 4096) + 1;   // + the plan block
     if (d.bf16)
         MLA_STEP_LAUNCH(q_rope_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, (const __nv_bfloat16 *)q,
-                        seq_lens, rows, s_q, d.H, d.d_r, d.d_n, d.base, (__nv_bfloat16 *)q_rot);
+                        seq_lens, rows, s_q, d.H, d.d_r, d.d_n, d.base, (__nv_bfloat16 *)q_rot, plan);
     else
         MLA_STEP_LAUNCH(q_rope_kernel<float>, dim3(blocks), dim3(256), 0, st, (const float *)q, seq_lens, rows, s_q,
-                        d.H, d.d_r, d.d_n, d.base, (float *)q_rot);
+                        d.H, d.d_r, d.d_n, d.base, (float *)q_rot, plan);
     return cudaGetLastError();
 }
 
@@ -136,8 +144,12 @@ __global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *
                                                            const __nv_bfloat16 *__restrict__ W_uk,
                                                            const int *__restrict__ seq_lens, int rows, int s_q,
                                                            int H, int hpw, float base,
-                                                           __nv_bfloat16 *__restrict__ q_abs) {
+                                                           __nv_bfloat16 *__restrict__ q_abs, PlanArgs plan) {
     step_begin();
+    if (blockIdx.x == H) {   // the extra column of blocks: its first block builds the split plan
+        if (blockIdx.y == 0 && blockIdx.z == 0) plan_block<256>(plan);
+        return;
+    }
     __shared__ __align__(16) __nv_bfloat16 As[AB_M * AB_LD];    // [64 rows][128 k]
     __shared__ __align__(16) __nv_bfloat16 Bs[AB_K * AB_LDB];   // [128 k][64 n]
     const int h = blockIdx.x, n0 = blockIdx.y * AB_N, row0 = blockIdx.z * AB_M;
@@ -209,11 +221,12 @@ __global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *
 bool q_absorb_mma_ok(const Dims &d) { return d.bf16 && d.d_n == 128 && d.d_c == 512 && d.d_r == 64; }
 
 cudaError_t launch_q_absorb_mma(const Dims &d, const void *q, const void *W_uk, const int *seq_lens, int batch,
-                                int s_q, void *q_abs, cudaStream_t st) {
+                                int s_q, void *q_abs, const PlanArgs &plan, cudaStream_t st) {
     const int rows = batch * s_q;
-    dim3 grid(d.H, 512 / AB_N, ceil_div(rows, AB_M));
+    dim3 grid(d.H + 1, 512 / AB_N, ceil_div(rows, AB_M));   // + one column for the plan block
     MLA_STEP_LAUNCH(q_absorb_mma_kernel, dim3(grid), dim3(256), 0, st, (const __nv_bfloat16 *)q,
-                    (const __nv_bfloat16 *)W_uk, seq_lens, rows, s_q, d.H, d.hpw, d.base, (__nv_bfloat16 *)q_abs);
+                    (const __nv_bfloat16 *)W_uk, seq_lens, rows, s_q, d.H, d.hpw, d.base, (__nv_bfloat16 *)q_abs,
+                    plan);
     return cudaGetLastError();
 }
 

@@ -316,13 +316,15 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
     void *qp = w + L.q_off;
     Plan plan{items, row_first, L.n_work, batch * L.plan_sq, L.chunk};
 
-    MLA_CUDA(launch_plan(seq_lens, batch, L.plan_sq, max_pages, d.page, L.chunk, L.n_work, items, row_first, err, st),
-             "launch plan");
+    const PlanArgs pa{seq_lens, batch, L.plan_sq, max_pages, d.page, L.chunk, L.n_work, items, row_first, err};
     if (path == ABSORBED) {
-        if (q_absorb_mma_ok(d))
-            MLA_CUDA(launch_q_absorb_mma(d, q, W_uk, seq_lens, batch, s_q, qp, st), "launch q_absorb (tensor cores)");
-        else
+        if (q_absorb_mma_ok(d)) {
+            MLA_CUDA(launch_q_absorb_mma(d, q, W_uk, seq_lens, batch, s_q, qp, pa, st),
+                     "launch q_absorb (tensor cores) + plan");
+        } else {
+            MLA_CUDA(launch_plan(pa, st), "launch plan");
             MLA_CUDA(launch_q_absorb(d, q, W_uk, seq_lens, batch, s_q, qp, st), "launch q_absorb");
+        }
         if (tc) {
             ProfileScope prof(st);
             MLA_CUDA(launch_tc_decode(d, qp, latent, page_table, plan, max_pages, n_pages, s_q, part_o, part_ml, err, sms,
@@ -341,7 +343,7 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
         else
             return fail(MLA_ERR_UNSUPPORTED, "tcgen05 partials need the tensor-core combine");
     } else {
-        MLA_CUDA(launch_q_rope(d, q, seq_lens, batch, s_q, qp, st), "launch q_rope");
+        MLA_CUDA(launch_q_rope(d, q, seq_lens, batch, s_q, qp, pa, st), "launch q_rope + plan");
         if (grouped_tc_ok(d, s_q)) {
             ProfileScope prof(st);
             MLA_CUDA(launch_grouped_decode(d, qp, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages,
@@ -499,9 +501,8 @@ mla_status mla_prefill_expanded(const mla_dims *dims, const void *q, const void 
     float *part_ml = (float *)(w + L.pml_off);
     void *qp = w + L.q_off;
     Plan plan{items, row_first, L.n_work, batch, L.chunk};
-    MLA_CUDA(launch_plan(seq_lens, batch, 1, max_pages, d.page, L.chunk, L.n_work, items, row_first, err, st),
-             "launch plan");
-    MLA_CUDA(launch_q_rope(d, q, seq_lens, batch, n_q, qp, st), "launch q_rope");
+    const PlanArgs pa{seq_lens, batch, 1, max_pages, d.page, L.chunk, L.n_work, items, row_first, err};
+    MLA_CUDA(launch_q_rope(d, q, seq_lens, batch, n_q, qp, pa, st), "launch q_rope + plan");
     {
         ProfileScope prof(st);
         MLA_CUDA(launch_prefill_expanded(d, qp, expanded_cache, latent_cache, seq_lens, page_table, plan, max_pages,

@@ -72,6 +72,15 @@ struct WorkItem {
     int split;   // chunk index inside the row
 };
 
+// Inputs and outputs of the device-side plan builder (plan_block.cuh).
+struct PlanArgs {
+    const int *seq_lens;
+    int batch, s_q, max_pages, page, chunk, n_expected;
+    WorkItem *items;     // [n_expected]
+    int *row_first;      // [batch * s_q + 1]
+    int *err;
+};
+
 struct Plan {
     const WorkItem *items;  // [n_work]
     const int *row_first;   // [rows + 1] first work item of each row (prefix sums)

@@ -28,10 +28,9 @@ cudaError_t launch_append_mma(const Dims &d, const void *h, int hidden, const vo
                               const int *req, const int *pos, int n_tok, const int *page_table, int batch,
                               int max_pages, int n_pages, void *cache, int *err, cudaStream_t st);
 
-// Split plan from device seq_lens (plan.cu).
-cudaError_t launch_plan(const int *seq_lens, int batch, int s_q, int max_pages, int page,
-                        int chunk, int n_work_expected, WorkItem *items, int *row_first,
-                        int *err, cudaStream_t st);
+// Split plan from device seq_lens as a kernel of its own (plan.cu).  launch_q_absorb_mma and
+// launch_q_rope build the same plan in an extra block instead.
+cudaError_t launch_plan(const PlanArgs &a, cudaStream_t st);
 
 // q absorption through W_UK + RoPE of the query's RoPE part (absorb.cu):
 //   q_abs [rows, H, d_c + d_r] = [W_UK[w]^T q_nope | RoPE(q_rope, p)], rows = batch * s_q.
@@ -40,12 +39,14 @@ cudaError_t launch_q_absorb(const Dims &d, const void *q, const void *W_uk, cons
 
 // Tensor-core variant for bf16, d_nope = 128, d_c = 512, d_rope = 64 (absorb.cu).
 bool q_absorb_mma_ok(const Dims &d);
+// It also builds the split plan `plan` in one extra block.
 cudaError_t launch_q_absorb_mma(const Dims &d, const void *q, const void *W_uk, const int *seq_lens, int batch,
-                                int s_q, void *q_abs, cudaStream_t st);
+                                int s_q, void *q_abs, const PlanArgs &plan, cudaStream_t st);
 
-// RoPE of the query's RoPE part only (absorb.cu): q_rot [rows, H, d_n + d_r].
+// RoPE of the query's RoPE part only (absorb.cu): q_rot [rows, H, d_n + d_r]; the split plan
+// `plan` is built in one extra block.
 cudaError_t launch_q_rope(const Dims &d, const void *q, const int *seq_lens, int batch, int s_q,
-                          void *q_rot, cudaStream_t st);
+                          void *q_rot, const PlanArgs &plan, cudaStream_t st);
 
 // General CUDA-core split flash decode (decode_simt.cu).  mode 0: absorbed (keys and values
 // are latent rows); mode 1: grouped (keys = [K_g | k_rope], values = V_g).

@@ -1,0 +1,87 @@
+// Split-KV plan built on the device by one thread block, from the device copy of seq_lens, so
+// that no host-to-device copy is needed per call.  Row r = (b, j) has len = seq_lens[b] - s_q +
+// j + 1 visible tokens, cut into ceil(len / chunk) chunks.  The host computes the same count
+// from its copy of seq_lens to size the grid and workspace; a disagreement (or a length outside
+// [s_q, max_pages * page]) sets MLA_ERR_INVALID_ARG and leaves an all-empty plan, so no kernel
+// reads or writes out of range.
+//
+// The block is either a kernel of its own (plan.cu) or one extra block of the query-preparation
+// kernel that runs before the decode, which saves a launch per call.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+// Run by all PT threads of one block (PT a multiple of 32, at most 1024).
+template <int PT>
+__device__ __forceinline__ void plan_block(const PlanArgs &a) {
+    static_assert(PT % 32 == 0 && PT <= 1024, "one warp scans the warp totals");
+    __shared__ int warp_sum[PT / 32];
+    __shared__ int bad;
+    const int rows = a.batch * a.s_q;
+    const int per = ceil_div(rows, PT);
+    const int r0 = min(rows, (int)threadIdx.x * per), r1 = min(rows, r0 + per);
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    if (threadIdx.x == 0) bad = 0;
+    __syncthreads();
+    int local = 0;
+    for (int r = r0; r < r1; ++r) {
+        const int b = r / a.s_q, j = r % a.s_q;
+        const int L = a.seq_lens[b];
+        if (L < a.s_q || L > a.max_pages * a.page) atomicOr(&bad, 1);
+        const int len = L - a.s_q + j + 1;
+        local += len > 0 ? ceil_div(len, a.chunk) : 0;
+    }
+    // Exclusive prefix of the per-thread counts: warp scans, then a scan of the warp totals.
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int w = lane < PT / 32 ? warp_sum[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, wi, off);
+            if (lane >= off) wi += v;
+        }
+        if (lane < PT / 32) warp_sum[lane] = wi - w;   // exclusive
+        if (lane == 31 && wi != a.n_expected) bad = 1;
+    }
+    __syncthreads();
+    const int first = warp_sum[warp] + incl - local;
+    if (bad) {
+        if (threadIdx.x == 0) report(a.err, MLA_ERR_INVALID_ARG);
+        for (int i = threadIdx.x; i < a.n_expected; i += PT) a.items[i] = WorkItem{0, 0, 0, 0};
+        for (int i = threadIdx.x; i <= rows; i += PT) a.row_first[i] = 0;
+        return;
+    }
+    int k = first;
+    for (int r = r0; r < r1; ++r) {
+        const int b = r / a.s_q, j = r % a.s_q;
+        a.row_first[r] = k;
+        k += ceil_div(a.seq_lens[b] - a.s_q + j + 1, a.chunk);
+    }
+    if (threadIdx.x == PT - 1) a.row_first[rows] = a.n_expected;
+    __syncthreads();   // row_first (global) is visible to the whole block after this barrier
+    // Items in parallel: item i belongs to the last row r with row_first[r] <= i.
+    for (int i = threadIdx.x; i < a.n_expected; i += PT) {
+        int lo = 0, hi = rows - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) / 2;
+            if (a.row_first[mid] <= i) lo = mid;
+            else hi = mid - 1;
+        }
+        const int b = lo / a.s_q, j = lo % a.s_q;
+        const int len = a.seq_lens[b] - a.s_q + j + 1;
+        const int c = i - a.row_first[lo];
+        a.items[i] = WorkItem{lo, c * a.chunk, min(len, (c + 1) * a.chunk), c};
+    }
+}
+
+}  // namespace mla
