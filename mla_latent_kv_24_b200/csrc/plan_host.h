@@ -1,4 +1,4 @@
-// Host side of the split-KV plan (the device side is plan.cu).  Both follow one rule:
+// Host side of the split-KV plan (the device side is plan_block.cuh).  Both follow one rule:
 // row (b, j) has len = seq_lens[b] - s_q + j + 1 tokens, cut into ceil(len / chunk) chunks.
 #pragma once
 
