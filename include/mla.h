@@ -21,7 +21,12 @@
  *     synchronises except in mla_get_device_status().  Scratch comes from a caller-provided
  *     workspace whose size the matching *_workspace_size() call returns.
  *   - Streams: work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
- *     and is asynchronous; argument errors are returned before anything is enqueued.
+ *     and is asynchronous; argument errors are returned before anything is enqueued.  The
+ *     kernels are launched with programmatic stream serialisation (programmatic dependent
+ *     launch): a kernel may be scheduled while the stream's previous kernel finishes, but it
+ *     waits for that kernel's completion before touching memory, so ordering against the
+ *     caller's own work on the stream is that of a plain stream.  Stream capture into a CUDA
+ *     graph records programmatic edges.
  *   - Layouts are row-major and densely packed unless stated.  bf16 = IEEE bfloat16 bits,
  *     fp32 = IEEE float.  All pointers of one call use the dtype in dims->dtype, except int32
  *     index arrays.  Device pointers must be 16-byte aligned.
