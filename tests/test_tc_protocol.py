@@ -1,0 +1,177 @@
+"""Model check of the tcgen05 absorbed decode's mbarrier protocol (decode_tc.cu), on CPU.
+
+Each role of the kernel (the K/Q producer, the V producer, the QK^T and PV issuers and the 16
+softmax warps of a CTA pair) is a coroutine that yields the barrier waits it performs, in the
+kernel's order, with the kernel's slot and parity arithmetic.  mbarriers follow the hardware's
+phase rule: a wait on parity P returns once the phase of that parity has completed, so a fresh
+barrier passes a wait on parity 1.  Every ring slot and buffer carries the generation its producer
+wrote, and every consumer asserts it reads the one it expects.  Random interleavings of the roles
+over random work-item lists must neither deadlock nor alias; planted mistakes must do one or the
+other, which shows the model can fail."""
+import random
+
+import pytest
+
+NK, NV = 3, 2              # K ring: three slots (one step); V ring: one slot per page of a step
+SOFTMAX_ARRIVALS = 16      # 8 softmax warps x 2 CTAs arrive on the counted barriers
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.phase = count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        if self.pending == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def passed(self, parity):
+        return (self.phase & 1) != parity
+
+
+def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=False):
+    """Runs the roles over work items (token steps per item) in a random order; returns "ok",
+    "deadlock", or raises AssertionError on a generation mismatch."""
+    rnd = random.Random(seed)
+    bars = {}
+
+    def bar(name, count=1):
+        return bars.setdefault(name, Bar(count))
+
+    for i in range(NK):
+        bar(("KFULL", i)), bar(("KEMPTY", i))
+    for i in range(NV):
+        bar(("VFULL", i)), bar(("VEMPTY", i))
+    bar("QFULL"), bar("QEMPTY")
+    for i in range(2):
+        bar(("SFULL", i)), bar(("SFREE", i), SOFTMAX_ARRIVALS), bar(("PVDONE", i))
+    bar("PFULL", SOFTMAX_ARRIVALS), bar("OFREE", SOFTMAX_ARRIVALS)
+    k_slots, v_slots, s_buf = [None] * NK, [None] * NV, [None, None]
+    state = {"Q": None, "P": None, "O": None}
+
+    def k_producer():
+        g = 0
+        for n, steps in enumerate(items):
+            if n > 0:
+                yield "QEMPTY", (n - 1) & 1
+            state["Q"] = n
+            bar("QFULL").arrive()
+            for _ in range(steps):
+                for j in range(NK):
+                    parity = (g & 1) ^ (0 if k_parity_flip else 1)
+                    yield ("KEMPTY", j), parity
+                    k_slots[j] = (g, j)
+                    bar(("KFULL", j)).arrive()
+                g += 1
+
+    def v_producer():
+        g = 0
+        for steps in items:
+            for _ in range(steps):
+                for pg in range(NV):
+                    yield ("VEMPTY", pg), (g & 1) ^ 1
+                    v_slots[pg] = (g, pg)
+                    bar(("VFULL", pg)).arrive()
+                g += 1
+
+    def qk_issuer():
+        g = 0
+        for n, steps in enumerate(items):
+            yield "QFULL", n & 1
+            for i in range(steps):
+                sb = g & 1
+                if g >= 2:
+                    yield ("SFREE", sb), ((g - 2) >> 1) & 1
+                for j in range(NK):
+                    yield ("KFULL", j), g & 1
+                    assert k_slots[j] == (g, j), ("K", k_slots[j], (g, j))
+                    assert state["Q"] == n, ("Q", state["Q"], n)
+                    bar(("KEMPTY", j)).arrive()
+                if i == steps - 1 and not skip_qempty:
+                    bar("QEMPTY").arrive()
+                s_buf[sb] = g
+                bar(("SFULL", sb)).arrive()
+                g += 1
+
+    def pv_issuer():
+        g = 0
+        for n, steps in enumerate(items):
+            for i in range(steps):
+                yield "PFULL", g & 1
+                if i == 0 and n > 0:
+                    yield "OFREE", (n - 1) & 1
+                assert state["P"] == g, ("P", state["P"], g)
+                for pg in range(NV):
+                    yield ("VFULL", pg), g & 1
+                    assert v_slots[pg] == (g, pg), ("V", v_slots[pg], (g, pg))
+                    bar(("VEMPTY", pg)).arrive()
+                state["O"] = n
+                bar(("PVDONE", g & 1)).arrive()
+                g += 1
+
+    def softmax_warp():
+        g = 0
+        for n, steps in enumerate(items):
+            for _ in range(steps):
+                sb = g & 1
+                yield ("SFULL", sb), (g >> 1) & 1
+                assert s_buf[sb] == g, ("S", s_buf[sb], g)
+                bar(("SFREE", sb)).arrive()
+                if g >= 1 and not skip_pv_wait:
+                    yield ("PVDONE", (g - 1) & 1), ((g - 1) >> 1) & 1
+                state["P"] = g
+                bar("PFULL").arrive()
+                g += 1
+            yield ("PVDONE", (g - 1) & 1), ((g - 1) >> 1) & 1
+            assert state["O"] == n, ("O", state["O"], n)
+            bar("OFREE").arrive()
+
+    roles = [k_producer(), v_producer(), qk_issuer(), pv_issuer()] + \
+        [softmax_warp() for _ in range(SOFTMAX_ARRIVALS)]
+    pending = {}
+    for r, co in enumerate(roles):
+        try:
+            pending[r] = next(co)
+        except StopIteration:
+            pass
+    while pending:
+        ready = [r for r, (name, parity) in pending.items() if bars[name].passed(parity)]
+        if not ready:
+            return "deadlock"
+        r = rnd.choice(ready)
+        try:
+            pending[r] = next(roles[r])
+        except StopIteration:
+            del pending[r]
+    return "ok"
+
+
+def _cases(n, seed0):
+    rnd = random.Random(seed0)
+    for s in range(n):
+        yield [rnd.randint(1, 6) for _ in range(rnd.randint(1, 4))], seed0 + s
+
+
+def test_protocol_has_no_deadlock_or_aliasing():
+    for items, seed in _cases(300, 1000):
+        assert simulate(items, seed) == "ok", (items, seed)
+
+
+def test_single_step_items_back_to_back():
+    # items of one step exercise the Q and O hand-over on every step
+    for seed in range(50):
+        assert simulate([1] * 6, seed) == "ok"
+
+
+# a wrong producer parity and a missing QEMPTY commit deadlock; writing P before PV(g-1) is done
+# lets PV(g-1) read P(g)
+@pytest.mark.parametrize("mistake", [dict(k_parity_flip=True), dict(skip_qempty=True), dict(skip_pv_wait=True)])
+def test_planted_mistakes_are_caught(mistake):
+    outcomes = set()
+    for items, seed in _cases(50, 2000):
+        try:
+            outcomes.add(simulate(items, seed, **mistake))
+        except AssertionError:
+            outcomes.add("alias")
+    assert outcomes & {"deadlock", "alias"}, outcomes
