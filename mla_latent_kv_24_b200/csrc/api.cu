@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -49,8 +50,11 @@ mla_status cuda_fail(cudaError_t e, const char *what) {
 }
 
 constexpr int MAX_DEVICES = 64;
-int *g_err_ptr[MAX_DEVICES];
-int g_sm_count[MAX_DEVICES];
+// Per-device constants, looked up on a device's first call.  The SM count is written before the
+// error-word pointer is published (release), and readers load the pointer first (acquire), so a
+// thread that sees the pointer also sees the count; concurrent first calls write the same values.
+std::atomic<int *> g_err_ptr[MAX_DEVICES];
+std::atomic<int> g_sm_count[MAX_DEVICES];
 
 // Device address of the error word and SM count of the current device, looked up once.
 mla_status device_info(int **err, int *sms) {
@@ -58,18 +62,20 @@ mla_status device_info(int **err, int *sms) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= MAX_DEVICES) return fail(MLA_ERR_UNSUPPORTED, "device ordinal %d too large", dev);
-    if (!g_err_ptr[dev]) {
+    int *ptr = g_err_ptr[dev].load(std::memory_order_acquire);
+    if (!ptr) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_device_error);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
         int n = 0;
         e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
-        g_sm_count[dev] = n;
-        g_err_ptr[dev] = (int *)p;
+        g_sm_count[dev].store(n, std::memory_order_relaxed);
+        ptr = (int *)p;
+        g_err_ptr[dev].store(ptr, std::memory_order_release);
     }
-    if (err) *err = g_err_ptr[dev];
-    if (sms) *sms = g_sm_count[dev];
+    if (err) *err = ptr;
+    if (sms) *sms = g_sm_count[dev].load(std::memory_order_relaxed);
     return MLA_OK;
 }
 
