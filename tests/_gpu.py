@@ -9,6 +9,10 @@ import workloads as wl
 # bf16 inputs, fp32 accumulation: normwise max relative error and mean absolute error.
 BF16_REL, BF16_MAE = 1e-2, 1e-3
 FP32_REL = 1e-5
+# Scale-free mean error for bf16: the GPU rounds q_abs, P and the output to bf16 (unit roundoff
+# 2^-9 each), which moves the mean relative error by a few 1e-3 at most; 1e-2 leaves a margin of
+# several times that while still failing a dropped term or a wrong index at any output scale.
+BF16_MAE_REL = 1e-2
 
 
 def dims_of(w: wl.Workload):
@@ -72,19 +76,43 @@ def prefill(dev: "Dev", expanded):
 
 def errors(got: np.ndarray, ref: np.ndarray):
     """(normwise max relative error, mean absolute error) over the finite entries of ref."""
+    f = figures(got, ref)
+    return f["rel"], f["mae"]
+
+
+def figures(got: np.ndarray, ref: np.ndarray) -> dict:
+    """Every error figure of one comparison, over the finite entries of ref:
+    rel       max|g - o| / max|o|              (normwise; gated in every test)
+    mae       mean|g - o|                      (absolute; gated for bf16)
+    mae_rel   mean|g - o| / mean|o|            (scale-free: at long contexts |o| is ~1e-3, where an
+                                                absolute MAE bound says little)
+    elem_max  max |g - o| / |o| over entries with |o| > 0.1 rms(o)   (element-wise, reported)
+    elem_p99  its 99th percentile                                      (reported)"""
     m = np.isfinite(ref)
-    g, r = got[m], ref[m]
+    g, r = got[m].astype(np.float64), ref[m].astype(np.float64)
     d = np.abs(g - r)
-    return float(d.max() / np.abs(r).max()), float(d.mean())
+    a = np.abs(r)
+    big = a > 0.1 * np.sqrt(np.mean(r * r))
+    el = d[big] / a[big] if big.any() else np.zeros(1)
+    return {"rel": float(d.max() / a.max()), "mae": float(d.mean()), "mae_rel": float(d.mean() / a.mean()),
+            "elem_max": float(el.max()), "elem_p99": float(np.percentile(el, 99)), "n": int(d.size)}
+
+
+# Figures of every comparison in this process, printed as a table at the end of the run.
+REPORT = []
 
 
 def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
     assert np.isfinite(got[np.isfinite(ref)]).all(), f"{what}: non-finite GPU output"
-    rel, mae = errors(got, ref)
+    f = figures(got, ref)
+    REPORT.append((what, dtype, f))
+    rel, mae = f["rel"], f["mae"]
+    msg = f"{what}: rel {rel:.3e} mae {mae:.3e} mae_rel {f['mae_rel']:.3e} elem_max {f['elem_max']:.3e}"
     if dtype == "bf16":
-        assert rel <= BF16_REL and mae <= BF16_MAE, f"{what}: rel {rel:.3e} mae {mae:.3e}"
+        assert rel <= BF16_REL and mae <= BF16_MAE, msg
+        assert f["mae_rel"] <= BF16_MAE_REL, msg
     else:
-        assert rel <= FP32_REL, f"{what}: rel {rel:.3e} mae {mae:.3e}"
+        assert rel <= FP32_REL, msg
     return rel, mae
 
 
