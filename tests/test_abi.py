@@ -97,3 +97,11 @@ def test_expand_tokens_argument_checks():
     assert lib.gqla_expand_tokens(ctypes.byref(d), 256, 256, 256, 256, 256, 4, 256, 0, 1, 1, 256, None) == 1
     assert lib.gqla_expand_tokens(ctypes.byref(d), 256, 256, 8, 256, 256, 4, 256, 1, 1, 1, 256, None) == 1
     assert "aligned" in mla.mla_last_error_string()
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    # The binding's copy of the static scratch size must be the header's, or the rejection test of
+    # the no-allocation entry point would probe the wrong bound.
+    m = re.search(r"#define\s+MLA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", open(HEADER).read())
+    assert m, "MLA_NOALLOC_SCRATCH_BYTES not found in include/mla.h"
+    assert int(m.group(1)) << int(m.group(2)) == mla.NOALLOC_SCRATCH_BYTES

@@ -55,6 +55,25 @@ def test_same_batch_twice_gives_the_same_output():
         assert rel <= BF16_REL and mae <= BF16_MAE, (rel, mae)
 
 
+def test_a_call_takes_no_device_memory():
+    # After a first call (which looks up the static scratch's address), a call with its output
+    # already allocated must leave the device's free memory exactly where it was.
+    w = wl.small_workload(wl.WORKLOADS["4"], B=3, s_q=2, lens=[900, 64, 2500], lens_loguniform=None, seed=35)
+    dev = Dev(wl.make_inputs(w))
+    out = torch.empty((w.B, w.s_q, w.H, w.d_v), dtype=dev.tdtype, device=dev.q.device)
+    call = lambda: mla.mla_decode_absorbed_noalloc(dev.dims, dev.q, dev.W_uk, dev.W_uv, dev.cache, dev.page_table,  # noqa: E731
+                                                   dev.seq_lens, dev.inp.seq_lens, w.B, w.s_q, dev.max_pages,
+                                                   dev.inp.n_pages, out)
+    call()
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    call()
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    mla.mla_get_device_status()
+    assert free_after == free_before, (free_before, free_after)
+
+
 def test_batch_too_large_for_the_static_scratch_is_rejected():
     w = wl.small_workload(wl.WORKLOADS["2"], B=1, lens=[64], seed=34)
     dev = Dev(wl.make_inputs(w))
