@@ -32,7 +32,7 @@
  *     index arrays.  Device pointers must be 16-byte aligned.
  *   - Positions: request b's cache holds seq_lens[b] tokens including its s_q current
  *     tokens (1 <= s_q <= 4: multi-token-prediction depth; the grouped tensor-core kernel
- *     covers s_q <= 2, deeper s_q runs the CUDA-core grouped decode);
+ *     holds 8 heads x 2 queries per 16-row tile and runs two tiles for s_q = 3, 4);
  *     query j (0 <= j < s_q) sits at position seq_lens[b] - s_q + j and attends to
  *     tokens t <= that position (this gives the causal mask between MTP query tokens).
  *     Token t of request b lives in page page_table[b*max_pages + t/page_size], row
@@ -42,6 +42,11 @@
  *     range, device seq_lens that contradict the host copy, a pipeline wait that ran out)
  *     set a per-device error word instead of faulting; the offending access is skipped and
  *     mla_get_device_status() reports it.
+ *   - Lifetime: on a device's first call the library looks up and keeps that device's address
+ *     of its error word and static scratch, and it keeps recent tensor-map encodings keyed by
+ *     buffer address.  These stay valid for the life of the device's primary context: do not
+ *     use the library across cudaDeviceReset() (or any teardown of the primary context) in
+ *     the same process.
  */
 #ifndef MLA_H_
 #define MLA_H_

@@ -15,11 +15,13 @@
 // each take 16 tokens of every 64-token page and keep their own online softmax; the CTA merges
 // the four (m, l, O) at the end and writes one partial result per query for the combine.
 //
-// The same kernel serves the head-expanded prefill path ("GQLA ..." abstract: MLA's absorbed
-// and head-expanded forms; the expanded form attends with K and V up-projected per head):
-// PREFILL CTAs take one head and 16 consecutive query tokens of a request (rows = queries),
-// read the per-head (heads_per_group = 1) or per-group expanded cache, and skip the pages that
-// lie after their last query's position (causal).
+// Deeper multi-token prediction (s_q = 3 or 4) uses two 16-row tiles (queries 0-1 and 2-3 of
+// the group's 8 heads): every K/V fragment a warp loads from shared memory feeds both tiles, so
+// the four queries still share each page read from HBM.
+//
+// The head-expanded prefill ("GQLA ..." abstract: MLA's absorbed and head-expanded forms) has
+// its own kernel below: one CTA per (head, 64-query tile), each warp owning 16 queries over all
+// tokens of the tile's causal range.
 #include <math.h>
 
 #include "tc_decode.h"
@@ -38,9 +40,10 @@ constexpr int WARPS = 4;
 constexpr int KV_TILE = PAGE * KV_LD, KR_TILE = PAGE * KR_LD;
 // The final cross-warp reduction reuses the stage buffers (all copies have landed by then).
 constexpr size_t STAGE_BYTES = sizeof(__nv_bfloat16) * STAGES * (KV_TILE + KR_TILE);
-constexpr size_t RED_BYTES = sizeof(float) * WARPS * 16 * (2 + D_V);
-static_assert(RED_BYTES <= STAGE_BYTES, "reduction buffer must fit in the stage buffers");
-constexpr size_t SMEM = STAGE_BYTES + sizeof(__nv_bfloat16) * 16 * Q_LD;   // 92416 B: 2 CTAs per SM
+constexpr size_t red_bytes(int rt) { return sizeof(float) * WARPS * 16 * rt * (2 + D_V); }
+static_assert(red_bytes(2) <= STAGE_BYTES, "reduction buffer must fit in the stage buffers");
+// 92416 B with one row tile, 98816 B with two: two CTAs per SM either way.
+constexpr size_t smem_bytes(int rt) { return STAGE_BYTES + sizeof(__nv_bfloat16) * 16 * rt * Q_LD; }
 
 struct GParams {
     const __nv_bfloat16 *q, *expanded, *latent;   // q: rotated queries [rows, H, 192]
@@ -52,41 +55,37 @@ struct GParams {
     int *err;
 };
 
-// Rows of the MMA tile.  Decode: CTA = (group g, item), row m = query m / 8 of head g*8 + m % 8.
-// Prefill: CTA = (head, item, query tile), row m = query 16 * tile + m of that head.
-template <bool PREFILL>
+// Rows of the MMA tiles: CTA = (group g, item), row m = query m / 8 of head g*8 + m % 8; RT row
+// tiles of 16 (RT = 1 for s_q <= 2, 2 for s_q = 3, 4).
+template <int RT>
 __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p) {
+    constexpr int ROWS = 16 * RT;
     step_begin();
     extern __shared__ __align__(16) uint8_t gsm[];
     __nv_bfloat16 *kv = reinterpret_cast<__nv_bfloat16 *>(gsm);           // [STAGES][64][KV_LD]
     __nv_bfloat16 *kr = kv + STAGES * KV_TILE;                            // [STAGES][64][KR_LD]
-    __nv_bfloat16 *qs = kr + STAGES * KR_TILE;                            // [16][Q_LD]
-    float *red_ml = reinterpret_cast<float *>(gsm);                       // [WARPS][16][2], after the loop
-    float *red_o = red_ml + WARPS * 16 * 2;                               // [WARPS][16][128], after the loop
+    __nv_bfloat16 *qs = kr + STAGES * KR_TILE;                            // [ROWS][Q_LD]
+    float *red_ml = reinterpret_cast<float *>(gsm);                       // [WARPS][ROWS][2], after the loop
+    float *red_o = red_ml + WARPS * ROWS * 2;                             // [WARPS][ROWS][128], after the loop
 
     // blockIdx.x = group (fastest), so the 16 groups of a chunk run together and the chunk's RoPE
     // keys, which every group reads, come from L2 after the first group's read.
-    const int item = PREFILL ? (int)blockIdx.y : (int)(blockIdx.z * 65535 + blockIdx.y);   // grid.y <= 65535
+    const int item = (int)(blockIdx.z * 65535 + blockIdx.y);   // grid.y <= 65535
     if (item >= p.plan.n_work) return;
     const WorkItem it = p.plan.items[item];
-    const int tile = PREFILL ? (int)blockIdx.z : 0;
-    const int head = blockIdx.x;                                  // prefill: the CTA's head
-    const int g = PREFILL ? head / p.hpw : (int)blockIdx.x;       // expanded-cache group
-    const int G = PREFILL ? p.H / p.hpw : p.H / GH;
-    auto row_query = [&](int m) { return PREFILL ? 16 * tile + m : m / GH; };
-    auto row_head = [&](int m) { return PREFILL ? head : g * GH + m % GH; };
+    const int g = (int)blockIdx.x;
+    const int G = p.H / GH;
+    auto row_query = [&](int m) { return m / GH; };
+    auto row_head = [&](int m) { return g * GH + m % GH; };
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int b = it.row;                   // the plan of this path has one row per request
     const int L = p.seq_lens[b];
-    // Prefill: pages after the tile's last query position are fully masked and are not read.
-    // Decode: every chunk ends at or before L, which the last query sees, so all its pages count.
-    const int last_q = min(p.s_q, row_query(15) + 1) - 1;
-    const int t_end = PREFILL ? min(it.t1, L - p.s_q + last_q + 1) : it.t1;
-    const int n_pg = PREFILL ? (t_end > it.t0 ? ceil_div(t_end - it.t0, PAGE) : 0) : ceil_div(it.t1 - it.t0, PAGE);
+    // Every chunk ends at or before L, which the last query sees, so all its pages count.
+    const int n_pg = ceil_div(it.t1 - it.t0, PAGE);
     const size_t part_base = (size_t)item * p.s_q;
 
     if (it.t1 <= it.t0) {   // only in a rejected plan
-        for (int m = tid; m < 16; m += blockDim.x) {
+        for (int m = tid; m < ROWS; m += blockDim.x) {
             if (row_query(m) >= p.s_q) continue;
             const size_t r = part_base + row_query(m);
             p.part_ml[(r * p.H + row_head(m)) * 2] = -INFINITY;
@@ -94,9 +93,9 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
         }
         return;
     }
-    // Queries, already rotated (q_rot = [q_nope | RoPE(q_rope, p_j)], one pass per call).  Decode:
-    // s_q = 2 fills all 16 rows, s_q = 1 the first 8; rows past the last query are zero.
-    for (int i = tid; i < 16 * (D_QK / 8); i += blockDim.x) {   // 16-byte chunks
+    // Queries, already rotated (q_rot = [q_nope | RoPE(q_rope, p_j)], one pass per call): s_q = 2
+    // fills the 16 rows of one tile, s_q = 1 the first 8; rows past the last query are zero.
+    for (int i = tid; i < ROWS * (D_QK / 8); i += blockDim.x) {   // 16-byte chunks
         const int m = i / (D_QK / 8), c = 8 * (i % (D_QK / 8));
         const int j = row_query(m), h = row_head(m);
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -130,23 +129,38 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
         }
     };
 
-    // Query A fragments stay in registers for the whole chunk (12 k-steps of 16 dims).
-    uint32_t qa[12][4];
+    // One tile's query A fragments stay in registers for the whole chunk (12 k-steps of 16 dims);
+    // with two tiles they are reloaded from shared memory per k-step (registers hold O instead).
+    uint32_t qa[RT == 1 ? 12 : 1][4];
+    if constexpr (RT == 1) {
 #pragma unroll
-    for (int ks = 0; ks < 12; ++ks)
-        ldmatrix_x4(qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3],
-                    qs + ((lane % 8) + 8 * ((lane / 8) % 2)) * Q_LD + 16 * ks + 8 * (lane / 16));
+        for (int ks = 0; ks < 12; ++ks)
+            ldmatrix_x4(qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3],
+                        qs + ((lane % 8) + 8 * ((lane / 8) % 2)) * Q_LD + 16 * ks + 8 * (lane / 16));
+    }
+    auto q_frag = [&](int t, int ks, uint32_t *f) {
+        ldmatrix_x4(f[0], f[1], f[2], f[3], qs + (16 * t + (lane % 8) + 8 * ((lane / 8) % 2)) * Q_LD + 16 * ks + 8 * (lane / 16));
+    };
 
     const int gid = lane / 4, t4 = lane % 4;
-    // Rows gid and gid + 8 of this thread's fragments: query index and visible length.
-    const int lim0 = row_query(gid) < p.s_q ? L - p.s_q + row_query(gid) : -1;
-    const int lim1 = row_query(gid + 8) < p.s_q ? L - p.s_q + row_query(gid + 8) : -1;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float o[16][4];
+    // Rows gid and gid + 8 of each tile's fragments: query index and last visible position.
+    int lim[RT][2];
+    float mrow[RT][2], lrow[RT][2];
+    float o[RT][16][4];
 #pragma unroll
-    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    for (int t = 0; t < RT; ++t) {
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int j = row_query(16 * t + gid + 8 * h2);
+            lim[t][h2] = j < p.s_q ? L - p.s_q + j : -1;
+            mrow[t][h2] = -INFINITY;
+            lrow[t][h2] = 0.f;
+        }
+#pragma unroll
+        for (int n = 0; n < 16; ++n) o[t][n][0] = o[t][n][1] = o[t][n][2] = o[t][n][3] = 0.f;
+    }
 
-    if (!PREFILL || n_pg > 0) load_page(0, 0);
+    load_page(0, 0);
     cp_async_commit();
     for (int i = 0; i < n_pg; ++i) {
         if (i + 1 < n_pg) load_page((i + 1) % STAGES, i + 1);
@@ -155,13 +169,245 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
         __syncthreads();
         const __nv_bfloat16 *tkv = kv + (i % STAGES) * KV_TILE + (16 * warp) * KV_LD;
         const __nv_bfloat16 *tkr = kr + (i % STAGES) * KR_TILE + (16 * warp) * KR_LD;
-        // S [16 rows x 16 tokens] = Q~ K~^T over 192 dims.
-        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // S [16 rows x 16 tokens] per tile = Q~ K~^T over 192 dims.
+        float s[RT][2][4];
+#pragma unroll
+        for (int t = 0; t < RT; ++t)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) s[t][nt][0] = s[t][nt][1] = s[t][nt][2] = s[t][nt][3] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < 12; ks += 2) {
+            uint32_t qf[RT][2][4];
+            if constexpr (RT > 1) {
+#pragma unroll
+                for (int t = 0; t < RT; ++t) {
+                    q_frag(t, ks, qf[t][0]);
+                    q_frag(t, ks + 1, qf[t][1]);
+                }
+            }
             // B fragments: rows = tokens, dims contiguous; x4 covers 2 k-steps of one n8 tile.
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
+                uint32_t bf[4];
+                const int tok = 8 * nt + (lane % 8);
+                const __nv_bfloat16 *src = ks < 8 ? tkv + tok * KV_LD + 16 * ks + 8 * (lane / 8)
+                                                  : tkr + tok * KR_LD + 16 * (ks - 8) + 8 * (lane / 8);
+                ldmatrix_x4(bf[0], bf[1], bf[2], bf[3], src);
+#pragma unroll
+                for (int t = 0; t < RT; ++t) {
+                    const uint32_t *a0 = RT == 1 ? qa[RT == 1 ? ks : 0] : qf[t][0];
+                    const uint32_t *a1 = RT == 1 ? qa[RT == 1 ? ks + 1 : 0] : qf[t][1];
+                    mma_bf16(s[t][nt], a0, bf[0], bf[1]);
+                    mma_bf16(s[t][nt], a1, bf[2], bf[3]);
+                }
+            }
+        }
+        // Mask, scale, online softmax per row (rows gid and gid + 8 of each tile; 4 tokens per row here).
+        const int tok_base = it.t0 + PAGE * i + 16 * warp;
+#pragma unroll
+        for (int t = 0; t < RT; ++t) {
+            float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int tk = tok_base + 8 * nt + 2 * t4 + e;
+                    const bool in = tk < it.t1;
+                    s[t][nt][e] = (in && tk <= lim[t][0]) ? s[t][nt][e] * p.scale_log2 : -INFINITY;
+                    s[t][nt][2 + e] = (in && tk <= lim[t][1]) ? s[t][nt][2 + e] * p.scale_log2 : -INFINITY;
+                    mx0 = fmaxf(mx0, s[t][nt][e]);
+                    mx1 = fmaxf(mx1, s[t][nt][2 + e]);
+                }
+#pragma unroll
+            for (int off = 1; off <= 2; off <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+            }
+            const float n0 = fmaxf(mrow[t][0], mx0), n1 = fmaxf(mrow[t][1], mx1);
+            const float a0 = n0 == -INFINITY ? 1.f : exp2f(mrow[t][0] - n0);
+            const float a1 = n1 == -INFINITY ? 1.f : exp2f(mrow[t][1] - n1);
+            float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    s[t][nt][e] = n0 == -INFINITY ? 0.f : exp2f(s[t][nt][e] - n0);
+                    s[t][nt][2 + e] = n1 == -INFINITY ? 0.f : exp2f(s[t][nt][2 + e] - n1);
+                    sum0 += s[t][nt][e];
+                    sum1 += s[t][nt][2 + e];
+                }
+            lrow[t][0] = lrow[t][0] * a0 + sum0;
+            lrow[t][1] = lrow[t][1] * a1 + sum1;
+            mrow[t][0] = n0;
+            mrow[t][1] = n1;
+#pragma unroll
+            for (int n = 0; n < 16; ++n) {
+                o[t][n][0] *= a0;
+                o[t][n][1] *= a0;
+                o[t][n][2] *= a1;
+                o[t][n][3] *= a1;
+            }
+        }
+        // P (accumulator layout of S) is the A fragment of P.V (rows x 16 tokens).
+        uint32_t pa[RT][4];
+#pragma unroll
+        for (int t = 0; t < RT; ++t) {
+            pa[t][0] = pack_bf16(s[t][0][0], s[t][0][1]);
+            pa[t][1] = pack_bf16(s[t][0][2], s[t][0][3]);
+            pa[t][2] = pack_bf16(s[t][1][0], s[t][1][1]);
+            pa[t][3] = pack_bf16(s[t][1][2], s[t][1][3]);
+        }
+        // O [16 x 128] += P V per tile: V rows = tokens with v contiguous; .trans gives B fragments,
+        // each shared by the tiles.
+#pragma unroll
+        for (int n = 0; n < 16; n += 2) {
+            uint32_t vb[4];
+            const __nv_bfloat16 *src = tkv + ((lane % 8) + 8 * ((lane / 8) % 2)) * KV_LD + D_N + 8 * n + 8 * (lane / 16);
+            ldmatrix_x4_trans(vb[0], vb[1], vb[2], vb[3], src);
+#pragma unroll
+            for (int t = 0; t < RT; ++t) {
+                mma_bf16(o[t][n], pa[t], vb[0], vb[1]);
+                mma_bf16(o[t][n + 1], pa[t], vb[2], vb[3]);
+            }
+        }
+        __syncthreads();   // this stage is refilled by the next iteration's load
+    }
+    cp_async_wait<0>();
+    __syncthreads();   // the stage buffers become the reduction buffer
+
+    // Merge the four warps' partial softmaxes: row sums over the 4 threads of each row first.
+#pragma unroll
+    for (int t = 0; t < RT; ++t)
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            float l = lrow[t][h2];
+#pragma unroll
+            for (int off = 1; off <= 2; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+            const int m = 16 * t + gid + 8 * h2;
+            if (t4 == 0) {
+                red_ml[(warp * ROWS + m) * 2] = mrow[t][h2];
+                red_ml[(warp * ROWS + m) * 2 + 1] = l;
+            }
+#pragma unroll
+            for (int n = 0; n < 16; ++n) {
+                red_o[(warp * ROWS + m) * D_V + 8 * n + 2 * t4] = o[t][n][2 * h2];
+                red_o[(warp * ROWS + m) * D_V + 8 * n + 2 * t4 + 1] = o[t][n][2 * h2 + 1];
+            }
+        }
+    __syncthreads();
+    // ROWS rows x 128 columns; rows past the last query are padding.
+    for (int i = tid; i < ROWS * D_V; i += blockDim.x) {
+        const int m = i / D_V, c = i % D_V, j = row_query(m);
+        if (j >= p.s_q) continue;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) M = fmaxf(M, red_ml[(w * ROWS + m) * 2]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) {
+            const float mw = red_ml[(w * ROWS + m) * 2];
+            const float wt = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            num += wt * red_o[(w * ROWS + m) * D_V + c];
+            den += wt * red_ml[(w * ROWS + m) * 2 + 1];
+        }
+        const size_t r = part_base + j;
+        const int h = row_head(m);
+        p.part_o[(r * p.H + h) * D_V + c] = num;   // relative to max M (log2 units)
+        if (c == 0) {
+            p.part_ml[(r * p.H + h) * 2] = M * 0.69314718055994531f;
+            p.part_ml[(r * p.H + h) * 2 + 1] = den;
+        }
+    }
+}
+
+
+// Head-expanded prefill: one CTA takes one head and PQ = 64 consecutive query tokens of one
+// request; warp w owns queries [16 w, 16 w + 16) of the tile over every token (the usual
+// flash-attention split), so each page of K|V and k^R is read once per 64 queries.  Pages after
+// the tile's last query position are skipped; the diagonal pages are masked per element.
+constexpr int PW = 4, PQ = 16 * PW;
+constexpr size_t P_SMEM = sizeof(__nv_bfloat16) * ((size_t)STAGES * (KV_TILE + KR_TILE) + (size_t)PQ * Q_LD);
+
+__global__ void __launch_bounds__(PW * 32, 2) prefill_kernel(GParams p) {
+    step_begin();
+    extern __shared__ __align__(16) uint8_t psm[];
+    __nv_bfloat16 *kv = reinterpret_cast<__nv_bfloat16 *>(psm);      // [STAGES][64][KV_LD]
+    __nv_bfloat16 *kr = kv + STAGES * KV_TILE;                         // [STAGES][64][KR_LD]
+    __nv_bfloat16 *qs = kr + STAGES * KR_TILE;                         // [PQ][Q_LD]
+    const int head = blockIdx.x, item = blockIdx.y, q0 = PQ * blockIdx.z;
+    if (item >= p.plan.n_work) return;
+    const WorkItem it = p.plan.items[item];
+    const int n_q = p.s_q;
+    const int g = head / p.hpw, G = p.H / p.hpw;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int b = it.row;
+    const int L = p.seq_lens[b];
+    const int q_last = min(n_q, q0 + PQ) - 1;
+    const int t_end = min(it.t1, L - n_q + q_last + 1);
+    const int n_pg = t_end > it.t0 ? ceil_div(t_end - it.t0, PAGE) : 0;
+    const size_t part_base = (size_t)item * n_q;
+
+    for (int i = tid; i < PQ * (D_QK / 8); i += blockDim.x) {   // 16-byte chunks of the query tile
+        const int m = i / (D_QK / 8), c = 8 * (i % (D_QK / 8)), q = q0 + m;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (q < n_q) v = *reinterpret_cast<const uint4 *>(p.q + (((size_t)b * n_q + q) * p.H + head) * D_QK + c);
+        *reinterpret_cast<uint4 *>(qs + m * Q_LD + c) = v;
+    }
+    auto load_page = [&](int stage, int i) {
+        int pid = p.page_table[(size_t)b * p.max_pages + it.t0 / PAGE + i];
+        bool ok = true;
+        if (pid < 0 || pid >= p.n_pages) {
+            if (tid == 0) report(p.err, MLA_ERR_DEVICE_BOUNDS);
+            ok = false;
+            pid = 0;
+        }
+        const int valid = ok ? min(PAGE, it.t1 - (it.t0 + PAGE * i)) : 0;
+        const __nv_bfloat16 *src_kv = p.expanded + (((size_t)pid * G + g) * PAGE) * 256;
+        const __nv_bfloat16 *src_kr = p.latent + ((size_t)pid * PAGE) * D_ROW + D_LAT;
+        __nv_bfloat16 *dkv = kv + stage * KV_TILE, *dkr = kr + stage * KR_TILE;
+        for (int c = tid; c < PAGE * 32; c += blockDim.x) {
+            const int r = c / 32, k = (c % 32) * 8;
+            cp_async16(dkv + r * KV_LD + k, src_kv + (size_t)r * 256 + k, r < valid);
+        }
+        for (int c = tid; c < PAGE * 8; c += blockDim.x) {
+            const int r = c / 8, k = (c % 8) * 8;
+            cp_async16(dkr + r * KR_LD + k, src_kr + (size_t)r * D_ROW + k, r < valid);
+        }
+    };
+    if (n_pg > 0) load_page(0, 0);
+    cp_async_commit();
+    __syncthreads();   // the query tile is in shared memory
+
+    uint32_t qa[12][4];
+#pragma unroll
+    for (int ks = 0; ks < 12; ++ks)
+        ldmatrix_x4(qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3],
+                    qs + (16 * warp + (lane % 8) + 8 * ((lane / 8) % 2)) * Q_LD + 16 * ks + 8 * (lane / 16));
+
+    const int gid = lane / 4, t4 = lane % 4;
+    const int qa0 = q0 + 16 * warp + gid, qa1 = qa0 + 8;          // this thread's two query rows
+    const int lim0 = qa0 < n_q ? L - n_q + qa0 : -1;              // last visible token of each
+    const int lim1 = qa1 < n_q ? L - n_q + qa1 : -1;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float o[16][4];
+#pragma unroll
+    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+
+    for (int i = 0; i < n_pg; ++i) {
+        if (i + 1 < n_pg) load_page((i + 1) % STAGES, i + 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        const __nv_bfloat16 *tkv = kv + (i % STAGES) * KV_TILE;
+        const __nv_bfloat16 *tkr = kr + (i % STAGES) * KR_TILE;
+        // S [16 rows x 64 tokens] = Q~ K~^T over 192 dims.
+        float s[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 12; ks += 2) {
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
                 uint32_t bf[4];
                 const int tok = 8 * nt + (lane % 8);
                 const __nv_bfloat16 *src = ks < 8 ? tkv + tok * KV_LD + 16 * ks + 8 * (lane / 8)
@@ -171,11 +417,10 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
                 mma_bf16(s[nt], qa[ks + 1], bf[2], bf[3]);
             }
         }
-        // Mask, scale, online softmax per row (rows gid and gid + 8; 4 tokens per row here).
-        const int tok_base = it.t0 + PAGE * i + 16 * warp;
+        const int tok_base = it.t0 + PAGE * i;
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int t = tok_base + 8 * nt + 2 * t4 + e;
@@ -194,7 +439,7 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
         const float a0 = n0 == -INFINITY ? 1.f : exp2f(m0 - n0), a1 = n1 == -INFINITY ? 1.f : exp2f(m1 - n1);
         float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 s[nt][e] = n0 == -INFINITY ? 0.f : exp2f(s[nt][e] - n0);
@@ -213,72 +458,49 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
             o[n][2] *= a1;
             o[n][3] *= a1;
         }
-        // P (accumulator layout of S) is the A fragment of P.V (rows x 16 tokens).
-        uint32_t pa[4] = {pack_bf16(s[0][0], s[0][1]), pack_bf16(s[0][2], s[0][3]), pack_bf16(s[1][0], s[1][1]),
-                          pack_bf16(s[1][2], s[1][3])};
-        // O [16 x 128] += P V: V rows = tokens with v contiguous; .trans gives B fragments.
+        // O [16 x 128] += P V, 16 tokens per k-step; P's accumulator layout is the A fragment.
 #pragma unroll
-        for (int n = 0; n < 16; n += 2) {
-            uint32_t vb[4];
-            const __nv_bfloat16 *src = tkv + ((lane % 8) + 8 * ((lane / 8) % 2)) * KV_LD + D_N + 8 * n + 8 * (lane / 16);
-            ldmatrix_x4_trans(vb[0], vb[1], vb[2], vb[3], src);
-            mma_bf16(o[n], pa, vb[0], vb[1]);
-            mma_bf16(o[n + 1], pa, vb[2], vb[3]);
+        for (int kt = 0; kt < 4; ++kt) {
+            const uint32_t pa[4] = {pack_bf16(s[2 * kt][0], s[2 * kt][1]), pack_bf16(s[2 * kt][2], s[2 * kt][3]),
+                                    pack_bf16(s[2 * kt + 1][0], s[2 * kt + 1][1]),
+                                    pack_bf16(s[2 * kt + 1][2], s[2 * kt + 1][3])};
+#pragma unroll
+            for (int n = 0; n < 16; n += 2) {
+                uint32_t vb[4];
+                const __nv_bfloat16 *src =
+                    tkv + (16 * kt + (lane % 8) + 8 * ((lane / 8) % 2)) * KV_LD + D_N + 8 * n + 8 * (lane / 16);
+                ldmatrix_x4_trans(vb[0], vb[1], vb[2], vb[3], src);
+                mma_bf16(o[n], pa, vb[0], vb[1]);
+                mma_bf16(o[n + 1], pa, vb[2], vb[3]);
+            }
         }
         __syncthreads();   // this stage is refilled by the next iteration's load
     }
     cp_async_wait<0>();
-    __syncthreads();   // the stage buffers become the reduction buffer
-
-    // Merge the four warps' partial softmaxes: row sums over the 4 threads of each row first.
 #pragma unroll
     for (int off = 1; off <= 2; off <<= 1) {
         l0 += __shfl_xor_sync(0xffffffffu, l0, off);
         l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
-    if (t4 == 0) {
-        red_ml[(warp * 16 + gid) * 2] = m0;
-        red_ml[(warp * 16 + gid) * 2 + 1] = l0;
-        red_ml[(warp * 16 + gid + 8) * 2] = m1;
-        red_ml[(warp * 16 + gid + 8) * 2 + 1] = l1;
-    }
+    // Each warp owns its rows: write the partial (relative to m, log2 units) and (m, l) directly.
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        red_o[(warp * 16 + gid) * D_V + 8 * n + 2 * t4] = o[n][0];
-        red_o[(warp * 16 + gid) * D_V + 8 * n + 2 * t4 + 1] = o[n][1];
-        red_o[(warp * 16 + gid + 8) * D_V + 8 * n + 2 * t4] = o[n][2];
-        red_o[(warp * 16 + gid + 8) * D_V + 8 * n + 2 * t4 + 1] = o[n][3];
-    }
-    __syncthreads();
-    // 16 rows x 128 columns; rows past the last query are padding.
-    for (int i = tid; i < 16 * D_V; i += blockDim.x) {
-        const int m = i / D_V, c = i % D_V, j = row_query(m);
-        if (j >= p.s_q) continue;
-        float M = -INFINITY;
+    for (int hr = 0; hr < 2; ++hr) {
+        const int q = hr ? qa1 : qa0;
+        if (q >= n_q) continue;
+        const size_t r = (part_base + q) * p.H + head;
 #pragma unroll
-        for (int w = 0; w < WARPS; ++w) M = fmaxf(M, red_ml[(w * 16 + m) * 2]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int w = 0; w < WARPS; ++w) {
-            const float mw = red_ml[(w * 16 + m) * 2];
-            const float wt = mw == -INFINITY ? 0.f : exp2f(mw - M);
-            num += wt * red_o[(w * 16 + m) * D_V + c];
-            den += wt * red_ml[(w * 16 + m) * 2 + 1];
-        }
-        const size_t r = part_base + j;
-        const int h = row_head(m);
-        p.part_o[(r * p.H + h) * D_V + c] = num;   // relative to max M (log2 units)
-        if (c == 0) {
-            p.part_ml[(r * p.H + h) * 2] = M * 0.69314718055994531f;
-            p.part_ml[(r * p.H + h) * 2 + 1] = den;
+        for (int n = 0; n < 16; ++n)
+            *reinterpret_cast<float2 *>(p.part_o + r * D_V + 8 * n + 2 * t4) = make_float2(o[n][2 * hr], o[n][2 * hr + 1]);
+        if (t4 == 0) {
+            p.part_ml[r * 2] = (hr ? m1 : m0) * 0.69314718055994531f;
+            p.part_ml[r * 2 + 1] = hr ? l1 : l0;
         }
     }
 }
-
 }  // namespace
 
 bool grouped_tc_ok(const Dims &d, int s_q) {
-    return s_q <= 2 && d.bf16 && d.hpw == GH && d.d_n == D_N && d.d_v == D_V && d.d_r == D_R && d.d_c == D_LAT && d.page == PAGE &&
+    return s_q <= 4 && d.bf16 && d.hpw == GH && d.d_n == D_N && d.d_v == D_V && d.d_r == D_R && d.d_c == D_LAT && d.page == PAGE &&
            d.H % GH == 0;
 }
 int grouped_units(const Dims &d, int sms) { return std::max(1, 8 * 2 * sms / std::max(1, d.H / GH)); }
@@ -312,10 +534,16 @@ cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expa
     if (plan.n_work == 0) return cudaSuccess;
     const GParams p = grouped_params(d, q, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages, s_q,
                                      part_o, part_ml, err);
-    cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<false>, SMEM);
-    if (e != cudaSuccess) return e;
     dim3 grid(d.H / GH, std::min(plan.n_work, 65535), ceil_div(plan.n_work, 65535));
-    MLA_STEP_LAUNCH(grouped_decode_kernel<false>, dim3(grid), dim3(WARPS * 32), SMEM, st, p);
+    if (s_q <= 2) {
+        cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<1>, smem_bytes(1));
+        if (e != cudaSuccess) return e;
+        MLA_STEP_LAUNCH(grouped_decode_kernel<1>, dim3(grid), dim3(WARPS * 32), smem_bytes(1), st, p);
+    } else {
+        cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<2>, smem_bytes(2));
+        if (e != cudaSuccess) return e;
+        MLA_STEP_LAUNCH(grouped_decode_kernel<2>, dim3(grid), dim3(WARPS * 32), smem_bytes(2), st, p);
+    }
     return cudaGetLastError();
 }
 
@@ -327,13 +555,13 @@ cudaError_t launch_prefill_expanded(const Dims &d, const void *q_rot, const void
                                     const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
                                     int n_pages, int n_q, float *part_o, float *part_ml, int *err, cudaStream_t st) {
     if (plan.n_work == 0) return cudaSuccess;
-    if (plan.n_work > 65535 || ceil_div(n_q, 16) > 65535) return cudaErrorInvalidValue;
+    if (plan.n_work > 65535 || ceil_div(n_q, PQ) > 65535) return cudaErrorInvalidValue;
     const GParams p = grouped_params(d, q_rot, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages, n_q,
                                      part_o, part_ml, err);
-    cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<true>, SMEM);
+    cudaError_t e = raise_smem_limit((const void *)prefill_kernel, P_SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid(d.H, plan.n_work, ceil_div(n_q, 16));
-    MLA_STEP_LAUNCH(grouped_decode_kernel<true>, dim3(grid), dim3(WARPS * 32), SMEM, st, p);
+    dim3 grid(d.H, plan.n_work, ceil_div(n_q, PQ));
+    MLA_STEP_LAUNCH(prefill_kernel, dim3(grid), dim3(PW * 32), P_SMEM, st, p);
     return cudaGetLastError();
 }
 

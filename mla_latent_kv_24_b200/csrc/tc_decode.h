@@ -15,7 +15,7 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
                              float *part_ml, int *err, int sms, cudaStream_t st);
 
 // Grouped path, bf16, d_nope = d_v = 128, d_rope = 64, heads_per_group = 8.
-bool grouped_tc_ok(const Dims &d, int s_q);   // s_q <= 2: one 16-row tile = 8 heads x 2 queries
+bool grouped_tc_ok(const Dims &d, int s_q);   // s_q <= 4: 16-row tiles of 8 heads x 2 queries
 int grouped_units(const Dims &d, int sms);
 int grouped_token_granule();
 // Head-expanded prefill over the expanded cache (per head with heads_per_group = 1, or per

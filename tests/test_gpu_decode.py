@@ -107,8 +107,8 @@ def test_grouped_ignores_nonfinite_stale_slots():
 
 @pytest.mark.parametrize("s_q", [3, 4])
 def test_deeper_mtp_both_paths_match_oracle(s_q):
-    # s_q = 3, 4: the absorbed path decodes every query row; the grouped path runs its CUDA-core
-    # decode (its tensor-core tile holds two queries).  One request has exactly s_q tokens.
+    # s_q = 3, 4: the absorbed path decodes every query row; the grouped path runs two 16-row
+    # tensor-core tiles (queries 0-1 and 2-3) over each K/V tile.  One request has exactly s_q tokens.
     w = wl.small_workload(wl.WORKLOADS["5_8192_1"], B=3, s_q=s_q, lens=[s_q, 130, 700], shuffle_pages=True,
                           seed=60 + s_q)
     inp = wl.make_inputs(w)
@@ -116,6 +116,24 @@ def test_deeper_mtp_both_paths_match_oracle(s_q):
     ref = oracle_decode(inp)
     assert_close(wl.from_torch_f64(dev.decode_absorbed()), ref, "bf16", f"absorbed s_q={s_q}")
     assert_close(wl.from_torch_f64(dev.decode_grouped(dev.expand())), ref, "bf16", f"grouped s_q={s_q}")
+
+
+@pytest.mark.parametrize("s_q,lens", [(4, (5000, 64)), (3, (129, 4097, 3)), (4, (4, 70, 2049, 1000))])
+def test_deeper_mtp_grouped_multi_chunk_matches_oracle(s_q, lens):
+    # long requests split into many chunks, some of which end between the queries' visible
+    # lengths; NaN in the stale slots of every last page must not reach the output
+    w = wl.small_workload(wl.WORKLOADS["5_8192_1"], B=len(lens), s_q=s_q, lens=list(lens), shuffle_pages=True,
+                          seed=90 + s_q + len(lens))
+    inp = wl.make_inputs(w)
+    dev = Dev(inp)
+    exp = dev.expand()
+    for b, L in enumerate(inp.seq_lens):
+        last = int(inp.page_table[b, (int(L) - 1) // w.page])
+        used = int(L) - ((int(L) - 1) // w.page) * w.page
+        exp[last, :, used:, :] = float("nan")
+        dev.cache.view(inp.n_pages, w.page, w.d_row)[last, used:, :] = float("nan")
+    assert_close(wl.from_torch_f64(dev.decode_grouped(exp)), oracle_decode(inp), "bf16",
+                 f"grouped s_q={s_q} multi-chunk {lens}")
 
 
 def test_deeper_mtp_mla_weights_match_oracle():
