@@ -15,7 +15,8 @@
 //   S  = Q K^T   M=128 heads, N=128 tokens, K=576: CTA r supplies the 64 tokens of page r of
 //                the step (B is split along N between the pair); S lands in 64 TMEM columns.
 //   O += P C     M=128 heads, N=256 latent columns (two instructions), K=128 tokens: CTA r
-//                supplies latent columns [256c + 128r, +128) of both pages.
+//                supplies latent columns [256c + 128r, +128) of both pages; P (the A operand)
+//                comes from tensor memory.
 // Every CTA loads only its own tiles, from its own GPU's HBM, with plain (non-multicast) TMA.
 //
 // Warp roles (384 threads per CTA): warps 0-7 softmax + epilogue (two warps per TMEM lane
@@ -24,16 +25,18 @@
 // warp 11 PV issuer (leader CTA only).  Shared memory holds Q
 // (72 KiB), a K ring of three 24 KiB slots (one step: the CTA's page x 576 columns as three
 // groups of three 64-column blocks), a V ring of two 32 KiB slots (one per page of the step:
-// this CTA's 256 latent columns) and one P tile.  Tiles move as few, large TMA boxes (3-D and
-// 4-D views of the [rows, 576] cache whose inner dimensions are 64-column blocks): a single
-// thread issuing one small box at a time cannot reach HBM bandwidth, while one instruction per
-// 24-32 KiB can.  K and V have separate rings and producers, so a V slot held until its PV
-// never stalls the next step's K loads.  (An L2 prefetch of the pages ahead of their K loads
-// was measured slower at every distance from one to four steps and is not used.)  S is
-// double-buffered in TMEM, so QK^T of step g+1 runs while the softmax of step g works.  The softmax rescales O only when a
-// row max grows by more than 2^8 (exact after the final division by l).  Every wait is bounded:
-// on timeout the kernel records MLA_ERR_TIMEOUT, stops issuing work, and still frees its
-// tensor memory before returning.
+// this CTA's 256 latent columns) and a 16 KiB buffer through which the softmax threads of lanes
+// L and L ^ 64 swap halves of P.  Tiles move as few, large TMA boxes (3-D and 4-D views of the
+// [rows, 576] cache whose inner dimensions are 64-column blocks): a single thread issuing one
+// small box at a time cannot reach HBM bandwidth, while one instruction per 24-32 KiB can.  K
+// and V have separate rings and producers, so a V slot held until its PV never stalls the next
+// step's K loads.  (An L2 prefetch of the pages ahead of their K loads was measured slower at
+// every distance from one to five steps and is not used.)  Tensor memory holds two S buffers
+// (QK^T of step g+1 runs while the softmax of step g works), O, and two P buffers (the softmax
+// of step g+1 writes P while PV of step g still reads the other one).  The softmax rescales O
+// only when a row max grows by more than 2^8 (exact after the final division by l), and only
+// then waits for the previous PV.  Every wait is bounded: on timeout the kernel records
+// MLA_ERR_TIMEOUT, stops issuing work, and still frees its tensor memory before returning.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -50,10 +53,10 @@ constexpr uint32_t BOX = 8192;                 // one 64-column block of 64 rows
 constexpr uint32_t KSLOT = 3 * BOX;
 constexpr uint32_t VSLOT = 4 * BOX;            // [chunk 0..1][block pair][64 rows][64 cols]
 constexpr uint32_t Q_BYTES = 9 * BOX;          // 64 heads x 576 bf16
-constexpr uint32_t P_BYTES = 2 * BOX;          // 64 heads x 128 tokens bf16
+constexpr uint32_t X_BYTES = 2 * BOX;          // P exchange: [2 column halves][128 lanes][64 B]
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_P = OFF_Q + Q_BYTES;
-constexpr uint32_t OFF_K = OFF_P + P_BYTES;
+constexpr uint32_t OFF_X = OFF_Q + Q_BYTES;
+constexpr uint32_t OFF_K = OFF_X + X_BYTES;
 constexpr uint32_t OFF_V = OFF_K + NK * KSLOT;
 constexpr uint32_t OFF_BAR = OFF_V + NV * VSLOT;
 enum {
@@ -66,7 +69,7 @@ enum {
     B_SFULL,
     B_SFREE = B_SFULL + 2,
     B_PFULL = B_SFREE + 2,
-    B_PVDONE,
+    B_PVDONE = B_PFULL + 2,
     B_OFREE = B_PVDONE + 2,
     B_COUNT
 };
@@ -81,6 +84,7 @@ static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 constexpr uint32_t TM_S = 0;      // two S buffers of 64 columns
 constexpr uint32_t TM_O = 128;    // O: 256 columns
+constexpr uint32_t TM_P = 384;    // two P buffers of 64 columns (bf16 pairs, duplicated lane halves)
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(128, 128, false, false);
@@ -240,7 +244,6 @@ __device__ void run_qk_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
 
 __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, int pair, int n_pairs) {
     int g = 0, item_n = 0;
-    const uint64_t pdesc = tc::sdesc_sw128(c.base + OFF_P, 16, 1024);
     const uint64_t vdesc = tc::sdesc_sw128(c.base + OFF_V, BOX, 1024);
     const uint32_t o_tmem = tmem + TM_O;
     for (int k = pair; k < p.plan.n_work; k += n_pairs) {
@@ -248,10 +251,11 @@ __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
         if (it.t1 <= it.t0) continue;
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
         for (int i = 0; i < n_steps; ++i, ++g) {
-            if (!wait_or_abort(c, c.bar(B_PFULL), (uint32_t)g & 1u, p.err)) return;
+            if (!wait_or_abort(c, c.bar(B_PFULL + (g & 1)), (uint32_t)(g >> 1) & 1u, p.err)) return;
             // The first PV of an item overwrites O: the previous item's epilogue must be done with it.
             if (i == 0 && item_n > 0 && !wait_or_abort(c, c.bar(B_OFREE), (uint32_t)(item_n - 1) & 1u, p.err)) return;
             tc::fence_after_sync();
+            const uint32_t p_tmem = tmem + TM_P + 64 * (g & 1);
 #pragma unroll
             for (int pg = 0; pg < NV; ++pg) {
                 if (!wait_or_abort(c, c.bar(B_VFULL + pg), (uint32_t)g & 1u, p.err)) return;
@@ -260,12 +264,12 @@ __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
                 for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
-                        const uint64_t a = tc::sdesc_add(pdesc, pg * BOX + 32 * k4);
+                        const uint32_t a = p_tmem + 32 * pg + 8 * k4;   // 16 tokens = 8 columns of bf16 pairs
                         const uint64_t bd = tc::sdesc_add(vdesc, pg * VSLOT + 2 * BOX * ch + 2048 * k4);
                         if (pg == 0 && k4 == 0 && i == 0)
-                            tc::mma_pair_bf16_k<false>(o_tmem + 128 * ch, a, bd, IDESC_PV);
+                            tc::mma_pair_ts_bf16_k<false>(o_tmem + 128 * ch, a, bd, IDESC_PV);
                         else
-                            tc::mma_pair_bf16_k<true>(o_tmem + 128 * ch, a, bd, IDESC_PV);
+                            tc::mma_pair_ts_bf16_k<true>(o_tmem + 128 * ch, a, bd, IDESC_PV);
                     }
                 tc::commit_pair(c.bar(B_VEMPTY + pg), 0x3);
             }
@@ -336,8 +340,12 @@ __device__ void run_softmax(const Ctx &c, const TcParams &p, uint32_t tmem, int 
             const float m_tile = fmaxf(fmaxf(mt, o1), fmaxf(o2, o3)) * p.scale_log2;   // head max, log2 units
             // One rescale decision for all heads keeps the tcgen05 loads below warp-uniform.
             const bool any = tc::named_sync_or(2, SM_THREADS, i > 0 && m_tile > m_run + RESCALE_LOG2);
-            // PV(g-1) must be complete before O is rescaled and before P is overwritten.
-            if (g >= 1) warp_wait(c, c.bar(B_PVDONE + ((g - 1) & 1)), (uint32_t)((g - 1) >> 1) & 1u, p.err);
+            // P is double-buffered: writing P(g) needs only PV(g-2) complete.  A rescale of O needs
+            // PV(g-1) complete (which implies PV(g-2)).  `any` is uniform over the CTA.
+            if (any && g >= 1)
+                warp_wait(c, c.bar(B_PVDONE + ((g - 1) & 1)), (uint32_t)((g - 1) >> 1) & 1u, p.err);
+            else if (g >= 2)
+                warp_wait(c, c.bar(B_PVDONE + (g & 1)), (uint32_t)((g - 2) >> 1) & 1u, p.err);
             tc::fence_after_sync();
             if (i == 0) {
                 m_run = m_tile;
@@ -370,16 +378,35 @@ __device__ void run_softmax(const Ctx &c, const TcParams &p, uint32_t tmem, int 
                 pk[j] = *reinterpret_cast<uint32_t *>(&h2);
             }
             l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-            uint8_t *prow = c.sbase + OFF_P + BOX * hsel + 128 * hl;
+            // P(g) into TMEM buffer g & 1 as the A operand of the two-CTA PV MMA, which takes the
+            // CTA's 64 rows twice (lanes L and L ^ 64 hold head L % 64 for all 128 tokens of the step;
+            // column c = tokens 2c, 2c + 1).  This thread has tokens [64 hsel + 32 half, +32), i.e.
+            // columns [32 hsel + 16 half, +16); the thread of lane L ^ 64 (warp w ^ 2, same half) has
+            // the other page's, swapped through shared memory.
+            {
+                uint4 *xb = reinterpret_cast<uint4 *>(c.sbase + OFF_X);   // [half][lane L][4 x 16 B]
+                const int sw = (lane >> 1) & 3;                          // conflict-free 16-byte slots
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                const uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-                *reinterpret_cast<uint4 *>(prow + (((4 * half + ch) ^ (hl & 7)) << 4)) = v;
+                for (int ch = 0; ch < 4; ++ch)
+                    xb[(128 * half + L) * 4 + (ch ^ sw)] = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+                tc::named_sync(3 + 2 * half + (warp & 1), 64);   // warps w and w ^ 2
+                uint32_t pp[16];
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const uint4 v = xb[(128 * half + (L ^ 64)) * 4 + (ch ^ sw)];
+                    pp[4 * ch] = v.x;
+                    pp[4 * ch + 1] = v.y;
+                    pp[4 * ch + 2] = v.z;
+                    pp[4 * ch + 3] = v.w;
+                }
+                const uint32_t pcol = tmem + TM_P + 64 * (g & 1) + 16 * half + lane_addr;
+                tc::tmem_st16(pcol + 32 * hsel, pk);
+                tc::tmem_st16(pcol + 32 * (hsel ^ 1), pp);
+                tc::tmem_wait_st();
             }
-            tc::fence_proxy_async_smem();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive_cluster(c.lead_bar(B_PFULL));
+            if (lane == 0) tc::mbar_arrive_cluster(c.lead_bar(B_PFULL + (g & 1)));
         }
         // Epilogue: the last PV of this item has landed; write the partial O, m, l.
         warp_wait(c, c.bar(B_PVDONE + ((g - 1) & 1)), (uint32_t)((g - 1) >> 1) & 1u, p.err);
@@ -449,6 +476,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tc::mbar_init(c.bar(B_PVDONE + i), 1);
         }
         tc::mbar_init(c.bar(B_PFULL), 2 * SOFTMAX_WARPS);
+        tc::mbar_init(c.bar(B_PFULL + 1), 2 * SOFTMAX_WARPS);
         tc::mbar_init(c.bar(B_OFREE), 2 * SOFTMAX_WARPS);
         *c.abort_flag = 0;
         tc::fence_mbar_init();

@@ -134,6 +134,20 @@ __device__ __forceinline__ void mma_pair_bf16_k(uint32_t d_tmem, uint64_t a_desc
                      "r"(idesc)
                      : "memory");
 }
+// Same with A read from tensor memory: each CTA's A rows at `a_tmem` in the layout the two-CTA
+// form takes for M = 128, the CTA's 64 rows in lanes 0-63 and again in lanes 64-127 (K pairs of
+// bf16 packed per 32-bit column).
+template <bool ACCUMULATE>
+__device__ __forceinline__ void mma_pair_ts_bf16_k(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc) {
+    if (ACCUMULATE)
+        asm volatile("tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, 1;" ::"r"(d_tmem), "r"(a_tmem),
+                     "l"(b_desc), "r"(idesc)
+                     : "memory");
+    else
+        asm volatile("tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, 0;" ::"r"(d_tmem), "r"(a_tmem),
+                     "l"(b_desc), "r"(idesc)
+                     : "memory");
+}
 // Arrive (once) on the barrier at this shared-memory offset in every CTA of `cta_mask` when
 // all previously issued MMAs of this thread complete.
 __device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t cta_mask) {
@@ -176,6 +190,15 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const float *v) {
         "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]),
         "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]),
         "r"(r[63])
+        : "memory");
+}
+// 32 lanes x 16 columns of 32-bit TMEM words from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
 // 32 lanes x 32 columns of 32-bit TMEM words.

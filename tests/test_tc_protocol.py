@@ -30,7 +30,12 @@ class Bar:
         return (self.phase & 1) != parity
 
 
-def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=False):
+def rescales(g):
+    """Steps whose softmax rescales O (a CTA-uniform decision in the kernel; here a fixed pattern)."""
+    return g % 5 == 3
+
+
+def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=False, skip_rescale_wait=False):
     """Runs the roles over work items (token steps per item) in a random order; returns "ok",
     "deadlock", or raises AssertionError on a generation mismatch."""
     rnd = random.Random(seed)
@@ -46,9 +51,9 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
     bar("QFULL"), bar("QEMPTY")
     for i in range(2):
         bar(("SFULL", i)), bar(("SFREE", i), SOFTMAX_ARRIVALS), bar(("PVDONE", i))
-    bar("PFULL", SOFTMAX_ARRIVALS), bar("OFREE", SOFTMAX_ARRIVALS)
-    k_slots, v_slots, s_buf = [None] * NK, [None] * NV, [None, None]
-    state = {"Q": None, "P": None, "O": None}
+    bar(("PFULL", 0), SOFTMAX_ARRIVALS), bar(("PFULL", 1), SOFTMAX_ARRIVALS), bar("OFREE", SOFTMAX_ARRIVALS)
+    k_slots, v_slots, s_buf, p_buf = [None] * NK, [None] * NV, [None, None], [None, None]
+    state = {"Q": None, "O": None, "pv_done": -1}
 
     def k_producer():
         g = 0
@@ -98,30 +103,37 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
         g = 0
         for n, steps in enumerate(items):
             for i in range(steps):
-                yield "PFULL", g & 1
+                yield ("PFULL", g & 1), (g >> 1) & 1
                 if i == 0 and n > 0:
                     yield "OFREE", (n - 1) & 1
-                assert state["P"] == g, ("P", state["P"], g)
+                assert p_buf[g & 1] == g, ("P", p_buf[g & 1], g)
                 for pg in range(NV):
                     yield ("VFULL", pg), g & 1
                     assert v_slots[pg] == (g, pg), ("V", v_slots[pg], (g, pg))
                     bar(("VEMPTY", pg)).arrive()
                 state["O"] = n
+                state["pv_done"] = g
                 bar(("PVDONE", g & 1)).arrive()
                 g += 1
 
     def softmax_warp():
         g = 0
         for n, steps in enumerate(items):
-            for _ in range(steps):
+            for i in range(steps):
                 sb = g & 1
                 yield ("SFULL", sb), (g >> 1) & 1
                 assert s_buf[sb] == g, ("S", s_buf[sb], g)
                 bar(("SFREE", sb)).arrive()
-                if g >= 1 and not skip_pv_wait:
+                # P is double-buffered: P(g) needs PV(g-2) done; a rescale of O needs PV(g-1) done
+                rescale = i > 0 and rescales(g)
+                if rescale and not skip_rescale_wait:
                     yield ("PVDONE", (g - 1) & 1), ((g - 1) >> 1) & 1
-                state["P"] = g
-                bar("PFULL").arrive()
+                elif g >= 2 and not skip_pv_wait:
+                    yield ("PVDONE", g & 1), ((g - 2) >> 1) & 1
+                if rescale:
+                    assert state["pv_done"] >= g - 1, ("rescale", state["pv_done"], g)
+                p_buf[g & 1] = g
+                bar(("PFULL", g & 1)).arrive()
                 g += 1
             yield ("PVDONE", (g - 1) & 1), ((g - 1) >> 1) & 1
             assert state["O"] == n, ("O", state["O"], n)
@@ -164,9 +176,10 @@ def test_single_step_items_back_to_back():
         assert simulate([1] * 6, seed) == "ok"
 
 
-# a wrong producer parity and a missing QEMPTY commit deadlock; writing P before PV(g-1) is done
-# lets PV(g-1) read P(g)
-@pytest.mark.parametrize("mistake", [dict(k_parity_flip=True), dict(skip_qempty=True), dict(skip_pv_wait=True)])
+# a wrong producer parity and a missing QEMPTY commit deadlock; writing P(g) before PV(g-2) is done
+# lets PV(g-2) read P(g); rescaling O before PV(g-1) is done races with it
+@pytest.mark.parametrize("mistake", [dict(k_parity_flip=True), dict(skip_qempty=True), dict(skip_pv_wait=True),
+                                     dict(skip_rescale_wait=True)])
 def test_planted_mistakes_are_caught(mistake):
     outcomes = set()
     for items, seed in _cases(50, 2000):
