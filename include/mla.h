@@ -149,9 +149,8 @@ MLA_API mla_status mla_decode_workspace_size(const mla_dims *dims, int32_t batch
  *   W_uk          device [H / heads_per_group, d_nope, d_c].
  *   W_uv          device [H / heads_per_group, d_v, d_c].
  *   latent_cache  device [n_pages_total, page_size, d_c + d_rope].  Slots past a request's
- *                 length in its last page must hold finite values (any finite values, e.g. a
- *                 zero-initialised pool): the tensor-core kernel multiplies their zero softmax
- *                 weights with them, and 0 * NaN would reach the output.
+ *                 length in its last page may hold anything, NaN included: they are never
+ *                 read into the softmax or the weighted sum.
  *   page_table    device [batch, max_pages];  seq_lens device [batch];
  *   seq_lens_host host   [batch], equal to the device copy; s_q <= seq_lens[b] <= max_pages*page.
  *   out           device [batch, s_q, H, d_v].
@@ -334,6 +333,20 @@ typedef enum { MLA_PATH_ABSORBED = 0, MLA_PATH_GROUPED = 1 } mla_path;
 MLA_API mla_status mla_select_path(const mla_dims *dims, int32_t batch, int32_t s_q, const int32_t *seq_lens_host,
                                    double hbm_bytes_per_s, double flops_per_s, int32_t tp, mla_path *path,
                                    double *t_absorbed_s, double *t_grouped_s);
+
+/*
+ * mla_debug_decode_fault — test hook of the bounded device waits (failure detection).  The
+ * pages have no counterpart to it.  After a call with withhold_step >= 0, every tensor-core
+ * absorbed decode launched from the calling thread skips the completion signal of pipeline
+ * step `withhold_step` (the PV product of that 128-token step) in every CTA pair, so the waits
+ * on it run out: the kernel records MLA_ERR_TIMEOUT in the device error word, stops issuing
+ * work, frees its tensor memory and returns without faulting; the call's output is garbage and
+ * mla_get_device_status() reports MLA_ERR_TIMEOUT.  wait_us (1..2000000) replaces the 2 s limit
+ * of every device wait, so the test ends in milliseconds; 0 keeps the default.
+ * mla_debug_decode_fault(-1, 0) restores normal operation.  Returns MLA_ERR_INVALID_ARG for
+ * withhold_step < -1 or wait_us > 2000000.  Not for production use.
+ */
+MLA_API mla_status mla_debug_decode_fault(int32_t withhold_step, uint32_t wait_us);
 
 /* Text of the last error on the calling thread ("" if none).  Valid until the next call. */
 MLA_API const char *mla_last_error_string(void);

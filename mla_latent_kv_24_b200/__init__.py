@@ -20,7 +20,7 @@ __all__ = [
     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
     "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
     "mla_decode_absorbed_noalloc", "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS", "mla_select_path",
-    "mla_prefill_workspace_size", "mla_prefill_expanded", "gqla_expand_tokens",
+    "mla_prefill_workspace_size", "mla_prefill_expanded", "gqla_expand_tokens", "mla_debug_decode_fault",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmla.so")
@@ -33,7 +33,7 @@ EXPORTED_SYMBOLS = ["mla_cache_append", "mla_decode_workspace_size", "mla_decode
                     "gqla_expand_cache", "gqla_decode_workspace_size", "gqla_decode_grouped",
                     "mla_get_device_status", "mla_last_error_string", "mla_version", "mla_set_profile_events",
                     "mla_decode_absorbed_noalloc", "mla_select_path", "mla_prefill_workspace_size",
-                    "mla_prefill_expanded", "gqla_expand_tokens"]
+                    "mla_prefill_expanded", "gqla_expand_tokens", "mla_debug_decode_fault"]
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -88,6 +88,7 @@ def load() -> ctypes.CDLL:
                             ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)],
         "mla_prefill_workspace_size": [D, _I, _I, _P, ctypes.POINTER(_S)],
         "mla_prefill_expanded": [D, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _S, _P],
+        "mla_debug_decode_fault": [_I, ctypes.c_uint32],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -234,3 +235,10 @@ def mla_prefill_expanded(dims, q, expanded_cache, latent_cache, page_table, seq_
     _check(load().mla_prefill_expanded(ctypes.byref(dims), _dev(q), _dev(expanded_cache), _dev(latent_cache),
                                        _dev(page_table), _dev(seq_lens), p, batch, n_q, max_pages, n_pages_total,
                                        _dev(out), _dev(workspace), nbytes, _stream(stream)))
+
+
+def mla_debug_decode_fault(withhold_step: int, wait_us: int = 0) -> None:
+    """Test hook: later tensor-core absorbed decodes on this thread withhold the completion signal
+    of pipeline step `withhold_step` (-1 restores normal operation) and give up every device wait
+    after `wait_us` microseconds (0: the 2 s default).  See include/mla.h."""
+    _check(load().mla_debug_decode_fault(withhold_step, wait_us))

@@ -233,6 +233,14 @@ mla_status mla_get_device_status(mla_stream_t stream) {
     return MLA_OK;
 }
 
+mla_status mla_debug_decode_fault(int32_t withhold_step, uint32_t wait_us) {
+    g_last_error.clear();
+    if (withhold_step < -1) return fail(MLA_ERR_INVALID_ARG, "withhold_step must be >= -1");
+    if (wait_us > 2000000u) return fail(MLA_ERR_INVALID_ARG, "wait_us must be <= 2000000");
+    tc_set_test_fault(withhold_step, (uint64_t)wait_us * 1000ull);
+    return MLA_OK;
+}
+
 mla_status mla_cache_append(const mla_dims *dims, const void *h, int32_t hidden, const void *W_dkv,
                             const void *W_kr, const int32_t *req_idx, const int32_t *positions, int32_t n_tok,
                             const int32_t *page_table, int32_t batch, int32_t max_pages, int32_t n_pages_total,

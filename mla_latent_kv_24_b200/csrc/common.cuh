@@ -60,6 +60,13 @@ __device__ __forceinline__ void step_begin() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// The split form, for kernels whose loads touch only the caller's inputs (weights, queries, hidden
+// states, lengths, page tables), which no kernel of this library writes: they let the next kernel
+// launch at once, load and compute while the previous kernel finishes, and call step_wait_prev()
+// before their first store.  Every thread that stores calls it, so the kernel completes only after
+// its predecessor has, and ordering down the stream stays that of a plain stream.
+__device__ __forceinline__ void step_allow_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void step_wait_prev() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------------------
 // Split-KV plan.  Row r = (b, j) has len_r = seq_lens[b] - s_q + j + 1 visible tokens and

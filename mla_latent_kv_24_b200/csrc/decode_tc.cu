@@ -71,6 +71,8 @@ enum {
     B_PFULL = B_SFREE + 2,
     B_PVDONE = B_PFULL + 2,
     B_OFREE = B_PVDONE + 2,
+    B_VLOCAL,   // this CTA's own copy of a ragged page's V tile (count 1, local)
+    B_VTAIL,    // both CTAs zeroed the stale rows of a ragged page's V tiles (count 2, leader)
     B_COUNT
 };
 constexpr uint32_t OFF_TMEMPTR = OFF_BAR + B_COUNT * 8;
@@ -105,6 +107,8 @@ struct TcParams {
     float *part_o;     // [n_work, 64, H, 8]: column octet-major (see the epilogue)
     float *part_ml;    // [n_work, H, 2]: max (natural-log units), sum
     int *err;
+    uint64_t wait_ns;  // limit of every barrier wait (WAIT_NS unless a test shortens it)
+    int withhold;      // test hook: the PV issuer skips the completion signal of this step (-1: none)
 };
 
 struct Ctx {
@@ -112,6 +116,7 @@ struct Ctx {
     uint8_t *sbase;     // generic pointer to the same
     uint32_t rank;      // 0 = leader of the pair
     volatile int *abort_flag;
+    uint64_t wait_ns;
     __device__ uint32_t bar(int i) const { return base + OFF_BAR + 8u * i; }
     __device__ uint32_t lead_bar(int i) const { return tc::map_to_rank(bar(i), 0); }
     __device__ uint32_t kslot(int i) const { return base + OFF_K + KSLOT * i; }
@@ -120,7 +125,7 @@ struct Ctx {
 
 __device__ __forceinline__ bool wait_or_abort(const Ctx &c, uint32_t bar, uint32_t parity, int *err) {
     if (*c.abort_flag) return false;
-    if (tc::mbar_wait(bar, parity, WAIT_NS)) return true;
+    if (tc::mbar_wait(bar, parity, c.wait_ns)) return true;
     report(err, MLA_ERR_TIMEOUT);
     *c.abort_flag = 1;
     return false;
@@ -177,7 +182,17 @@ __device__ void run_k_producer(const Ctx &c, const TcParams &p, const CUtensorMa
     }
 }
 
-// V producer: per step and page pg of the step, this CTA's 256 latent columns of that page.
+// Rows of the page starting at token `row0` that lie inside the item, when that is a proper part
+// of the page (the request's ragged last page): its other rows are slots past the request's length,
+// which may hold anything, NaN included.  0 otherwise.
+__device__ __forceinline__ int ragged_rows(const WorkItem &it, int row0) {
+    const int valid = it.t1 - row0;
+    return (valid > 0 && valid < PAGE) ? valid : 0;
+}
+
+// V producer (lane 0): per step and page pg of the step, this CTA's 256 latent columns of that
+// page.  A ragged page is copied with this CTA's own barrier instead, and its stale rows are
+// cleared by run_v_tail.
 __device__ void run_v_producer(const Ctx &c, const TcParams &p, const CUtensorMap *tm_v, int pair, int n_pairs) {
     int g = 0;
     for (int k = pair; k < p.plan.n_work; k += n_pairs) {
@@ -190,10 +205,48 @@ __device__ void run_v_producer(const Ctx &c, const TcParams &p, const CUtensorMa
             for (int pg = 0; pg < NV; ++pg) {
                 const int y = page_row(p, b, t_step / PAGE + pg, it.t1);
                 if (!wait_or_abort(c, c.bar(B_VEMPTY + pg), ((uint32_t)g & 1u) ^ 1u, p.err)) return;
-                if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_VFULL + pg), 2u * VSLOT);
-                tc::tma_load_4d_pair(c.vslot(pg), tm_v, 0, y, 2 * (int)c.rank, 0, c.lead_bar(B_VFULL + pg));
+                if (!ragged_rows(it, t_step + PAGE * pg)) {
+                    if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_VFULL + pg), 2u * VSLOT);
+                    tc::tma_load_4d_pair(c.vslot(pg), tm_v, 0, y, 2 * (int)c.rank, 0, c.lead_bar(B_VFULL + pg));
+                } else {
+                    // This phase of VFULL carries no bytes; the PV issuer waits on the tail barrier.
+                    if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_VFULL + pg), 0u);
+                    tc::mbar_arrive_expect_tx(c.bar(B_VLOCAL), VSLOT);
+                    tc::tma_load_4d(c.vslot(pg), tm_v, 0, y, 2 * (int)c.rank, 0, c.bar(B_VLOCAL));
+                }
             }
         }
+    }
+}
+
+// Lanes 1-31 of the V producer's warp: for each ragged page, once its copy has landed, zero the
+// rows past the item's end in this CTA's V tile (their probabilities are zero, but 0 x NaN is
+// NaN in P.V), make the stores visible to the tensor core and report on the leader's tail
+// barrier.  Zeroing whole 128-byte rows of each 64-column block needs no knowledge of the
+// 128-byte swizzle.
+__device__ void run_v_tail(const Ctx &c, const TcParams &p, int pair, int n_pairs) {
+    const int lane = threadIdx.x % 32;   // 1..31
+    int nt = 0;                          // ragged pages so far (phase of B_VLOCAL)
+    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
+        const WorkItem it = p.plan.items[k];
+        if (it.t1 <= it.t0) continue;
+        const int n_steps = ceil_div(it.t1 - it.t0, STEP);
+        for (int i = n_steps - 1; i < n_steps; ++i)   // only an item's last step can hold its end
+            for (int pg = 0; pg < NV; ++pg) {
+                const int valid = ragged_rows(it, it.t0 + STEP * i + PAGE * pg);
+                if (!valid) continue;
+                const bool ok = wait_or_abort(c, c.bar(B_VLOCAL), (uint32_t)(nt++) & 1u, p.err);
+                if (!__all_sync(0xfffffffeu, ok)) return;
+                uint8_t *tile = c.sbase + OFF_V + VSLOT * pg;      // four [64 rows][128 B] blocks
+                const int n16 = (PAGE - valid) * 8;                // 16-byte pieces past the end, per block
+                for (int e = lane - 1; e < 4 * n16; e += 31) {
+                    const int blk = e / n16, r = e % n16;
+                    *reinterpret_cast<uint4 *>(tile + BOX * blk + 128 * valid + 16 * r) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                tc::fence_proxy_async_smem();
+                __syncwarp(0xfffffffeu);
+                if (lane == 1) tc::mbar_arrive_cluster(c.lead_bar(B_VTAIL));
+            }
     }
 }
 
@@ -243,7 +296,7 @@ __device__ void run_qk_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
 }
 
 __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, int pair, int n_pairs) {
-    int g = 0, item_n = 0;
+    int g = 0, item_n = 0, nt = 0;   // nt: ragged pages so far (phase of B_VTAIL)
     const uint64_t vdesc = tc::sdesc_sw128(c.base + OFF_V, BOX, 1024);
     const uint32_t o_tmem = tmem + TM_O;
     for (int k = pair; k < p.plan.n_work; k += n_pairs) {
@@ -259,6 +312,9 @@ __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
 #pragma unroll
             for (int pg = 0; pg < NV; ++pg) {
                 if (!wait_or_abort(c, c.bar(B_VFULL + pg), (uint32_t)g & 1u, p.err)) return;
+                if (ragged_rows(it, it.t0 + STEP * i + PAGE * pg) &&
+                    !wait_or_abort(c, c.bar(B_VTAIL), (uint32_t)(nt++) & 1u, p.err))
+                    return;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int ch = 0; ch < 2; ++ch)
@@ -273,7 +329,7 @@ __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
                     }
                 tc::commit_pair(c.bar(B_VEMPTY + pg), 0x3);
             }
-            tc::commit_pair(c.bar(B_PVDONE + (g & 1)), 0x3);
+            if (g != p.withhold) tc::commit_pair(c.bar(B_PVDONE + (g & 1)), 0x3);
         }
         ++item_n;
     }
@@ -443,7 +499,9 @@ __device__ void run_softmax(const Ctx &c, const TcParams &p, uint32_t tmem, int 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, TcParams p) {
-    step_begin();
+    // Barrier set-up and the tensor-memory allocation touch no global memory: they run while the
+    // previous kernel (the query absorption) finishes; the roles start after step_wait_prev().
+    step_allow_next();
     extern __shared__ uint8_t smem_raw[];
     Ctx c;
     const uint32_t raw = tc::smem_addr(smem_raw);
@@ -451,10 +509,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     c.sbase = smem_raw + (c.base - raw);
     c.rank = tc::cluster_rank();
     c.abort_flag = reinterpret_cast<volatile int *>(c.sbase + OFF_FLAG);
+    c.wait_ns = p.wait_ns;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     uint32_t dyn_bytes;
     asm("mov.u32 %0, %dynamic_smem_size;" : "=r"(dyn_bytes));
     if (c.base - raw + SMEM_USED > dyn_bytes) {   // uniform for the whole cluster: nothing ran yet
+        step_wait_prev();
         if (threadIdx.x == 0) report(p.err, MLA_ERR_UNSUPPORTED);
         return;
     }
@@ -478,6 +538,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc::mbar_init(c.bar(B_PFULL), 2 * SOFTMAX_WARPS);
         tc::mbar_init(c.bar(B_PFULL + 1), 2 * SOFTMAX_WARPS);
         tc::mbar_init(c.bar(B_OFREE), 2 * SOFTMAX_WARPS);
+        tc::mbar_init(c.bar(B_VLOCAL), 1);
+        tc::mbar_init(c.bar(B_VTAIL), 2);
         *c.abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -492,12 +554,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc::cluster_sync();
     tc::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(c.sbase + OFF_TMEMPTR);
+    step_wait_prev();   // q_abs and the plan come from the previous kernel
 
     const int pair = blockIdx.x / 2, n_pairs = gridDim.x / 2;
     if (warp == W_KPROD) {
         if (lane == 0) run_k_producer(c, p, &tm_q, &tm_k, pair, n_pairs);
     } else if (warp == W_VPROD) {
-        if (lane == 0) run_v_producer(c, p, &tm_v, pair, n_pairs);
+        if (lane == 0)
+            run_v_producer(c, p, &tm_v, pair, n_pairs);
+        else
+            run_v_tail(c, p, pair, n_pairs);
     } else if (warp == W_MMA) {
         if (c.rank == 0 && lane == 0) run_qk_issuer(c, p, tmem, pair, n_pairs);
     } else if (warp == W_PV) {
@@ -595,7 +661,15 @@ bool encode_blocks_cached(CUtensorMap *m, const void *ptr, uint64_t rows, int nb
     return true;
 }
 
+thread_local int g_test_withhold = -1;
+thread_local uint64_t g_test_wait_ns = WAIT_NS;
+
 }  // namespace
+
+void tc_set_test_fault(int withhold_step, uint64_t wait_ns) {
+    g_test_withhold = withhold_step < 0 ? -1 : withhold_step;
+    g_test_wait_ns = wait_ns == 0 ? WAIT_NS : wait_ns;
+}
 
 bool tc_available() { return true; }
 int tc_units(int sms) { return sms / 2; }
@@ -620,6 +694,8 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
     p.part_o = part_o;
     p.part_ml = part_ml;
     p.err = err;
+    p.wait_ns = g_test_wait_ns;
+    p.withhold = g_test_withhold;
     cudaError_t e = raise_smem_limit((const void *)tc_decode_kernel, SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     const int units = std::max(1, std::min(plan.n_work, std::max(1, sms / 2)));

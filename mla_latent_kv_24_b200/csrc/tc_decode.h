@@ -14,6 +14,11 @@ cudaError_t launch_tc_decode(const Dims &d, const void *q_abs, const void *laten
                              const Plan &plan, int max_pages, int n_pages, int s_q, float *part_o,
                              float *part_ml, int *err, int sms, cudaStream_t st);
 
+// Test hook of the bounded waits: later tcgen05 decodes on the calling thread skip the completion
+// signal of pipeline step `withhold_step` (-1: none) and give up every wait after `wait_ns`
+// (0: the default 2 s).
+void tc_set_test_fault(int withhold_step, uint64_t wait_ns);
+
 // Grouped path, bf16, d_nope = d_v = 128, d_rope = 64, heads_per_group = 8.
 bool grouped_tc_ok(const Dims &d, int s_q);   // s_q <= 4: 16-row tiles of 8 heads x 2 queries
 int grouped_units(const Dims &d, int sms);

@@ -105,3 +105,11 @@ def test_noalloc_scratch_size_matches_the_header():
     m = re.search(r"#define\s+MLA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", open(HEADER).read())
     assert m, "MLA_NOALLOC_SCRATCH_BYTES not found in include/mla.h"
     assert int(m.group(1)) << int(m.group(2)) == mla.NOALLOC_SCRATCH_BYTES
+
+
+def test_debug_fault_hook_argument_checks():
+    # thread-local host state only: no device is touched
+    assert mla.load().mla_debug_decode_fault(-2, 0) == 1
+    assert mla.load().mla_debug_decode_fault(0, 2000001) == 1
+    mla.mla_debug_decode_fault(3, 1000)
+    mla.mla_debug_decode_fault(-1, 0)

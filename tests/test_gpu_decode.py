@@ -105,6 +105,23 @@ def test_grouped_ignores_nonfinite_stale_slots():
     assert_close(got, oracle_decode(inp), "bf16", "grouped with NaN stale slots")
 
 
+@pytest.mark.parametrize("s_q,lens", [(1, (70, 130, 1000, 64)), (2, (70, 129, 1000, 5))])
+def test_absorbed_ignores_nonfinite_stale_slots(s_q, lens):
+    # slots past a request's length in its last page hold NaN; the tensor-core kernel loads whole
+    # pages, so it must clear those rows before P.V (a zero probability times NaN is NaN)
+    w = wl.small_workload(wl.WORKLOADS["4"], B=len(lens), s_q=s_q, lens=list(lens), lens_loguniform=None,
+                          shuffle_pages=True, seed=23 + s_q)
+    inp = wl.make_inputs(w)
+    dev = Dev(inp)
+    for b, L in enumerate(inp.seq_lens):
+        last = int(inp.page_table[b, (int(L) - 1) // w.page])
+        used = int(L) - ((int(L) - 1) // w.page) * w.page
+        dev.cache.view(inp.n_pages, w.page, w.d_row)[last, used:, :] = float("nan")
+    got = wl.from_torch_f64(dev.decode_absorbed())
+    mla.mla_get_device_status()
+    assert_close(got, oracle_decode(inp), "bf16", f"absorbed with NaN stale slots s_q={s_q}")
+
+
 @pytest.mark.parametrize("s_q", [3, 4])
 def test_deeper_mtp_both_paths_match_oracle(s_q):
     # s_q = 3, 4: the absorbed path decodes every query row; the grouped path runs two 16-row

@@ -35,7 +35,14 @@ def rescales(g):
     return g % 5 == 3
 
 
-def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=False, skip_rescale_wait=False):
+def ragged(n, steps, pg):
+    """Whether page pg of the last step of item n is a request's ragged last page (a fixed pattern;
+    the kernel decides it from the item's end)."""
+    return (n % 3 == 1 and pg == 1) or (n % 3 == 2 and pg == 0 and steps % 2 == 0)
+
+
+def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=False, skip_rescale_wait=False,
+             skip_tail_wait=False):
     """Runs the roles over work items (token steps per item) in a random order; returns "ok",
     "deadlock", or raises AssertionError on a generation mismatch."""
     rnd = random.Random(seed)
@@ -52,6 +59,7 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
     for i in range(2):
         bar(("SFULL", i)), bar(("SFREE", i), SOFTMAX_ARRIVALS), bar(("PVDONE", i))
     bar(("PFULL", 0), SOFTMAX_ARRIVALS), bar(("PFULL", 1), SOFTMAX_ARRIVALS), bar("OFREE", SOFTMAX_ARRIVALS)
+    bar("VTAIL")
     k_slots, v_slots, s_buf, p_buf = [None] * NK, [None] * NV, [None, None], [None, None]
     state = {"Q": None, "O": None, "pv_done": -1}
 
@@ -72,12 +80,21 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
 
     def v_producer():
         g = 0
-        for steps in items:
-            for _ in range(steps):
+        for n, steps in enumerate(items):
+            for i in range(steps):
                 for pg in range(NV):
                     yield ("VEMPTY", pg), (g & 1) ^ 1
-                    v_slots[pg] = (g, pg)
-                    bar(("VFULL", pg)).arrive()
+                    if i == steps - 1 and ragged(n, steps, pg):
+                        # the copy lands on the CTA's own barrier; VFULL's phase carries no bytes, and
+                        # the tile is complete (stale rows zeroed) only at the tail barrier
+                        v_slots[pg] = "partial"
+                        bar(("VFULL", pg)).arrive()
+                        yield None, None                 # the copy and the zeroing take a while
+                        v_slots[pg] = (g, pg)
+                        bar("VTAIL").arrive()
+                    else:
+                        v_slots[pg] = (g, pg)
+                        bar(("VFULL", pg)).arrive()
                 g += 1
 
     def qk_issuer():
@@ -101,6 +118,7 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
 
     def pv_issuer():
         g = 0
+        nt = 0
         for n, steps in enumerate(items):
             for i in range(steps):
                 yield ("PFULL", g & 1), (g >> 1) & 1
@@ -109,6 +127,10 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
                 assert p_buf[g & 1] == g, ("P", p_buf[g & 1], g)
                 for pg in range(NV):
                     yield ("VFULL", pg), g & 1
+                    if i == steps - 1 and ragged(n, steps, pg):
+                        if not skip_tail_wait:
+                            yield "VTAIL", nt & 1
+                        nt += 1
                     assert v_slots[pg] == (g, pg), ("V", v_slots[pg], (g, pg))
                     bar(("VEMPTY", pg)).arrive()
                 state["O"] = n
@@ -148,7 +170,7 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
         except StopIteration:
             pass
     while pending:
-        ready = [r for r, (name, parity) in pending.items() if bars[name].passed(parity)]
+        ready = [r for r, (name, parity) in pending.items() if name is None or bars[name].passed(parity)]
         if not ready:
             return "deadlock"
         r = rnd.choice(ready)
@@ -177,9 +199,10 @@ def test_single_step_items_back_to_back():
 
 
 # a wrong producer parity and a missing QEMPTY commit deadlock; writing P(g) before PV(g-2) is done
-# lets PV(g-2) read P(g); rescaling O before PV(g-1) is done races with it
+# lets PV(g-2) read P(g); rescaling O before PV(g-1) is done races with it; reading a ragged V tile
+# before its tail barrier sees its stale rows
 @pytest.mark.parametrize("mistake", [dict(k_parity_flip=True), dict(skip_qempty=True), dict(skip_pv_wait=True),
-                                     dict(skip_rescale_wait=True)])
+                                     dict(skip_rescale_wait=True), dict(skip_tail_wait=True)])
 def test_planted_mistakes_are_caught(mistake):
     outcomes = set()
     for items, seed in _cases(50, 2000):
