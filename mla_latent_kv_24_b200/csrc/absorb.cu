@@ -67,7 +67,8 @@ __global__ void __launch_bounds__(256) q_rope_kernel(const T *__restrict__ q, co
                                                      T *__restrict__ q_rot, PlanArgs plan) {
     step_begin();
     if (blockIdx.x == gridDim.x - 1) {
-        plan_block<256>(plan);
+        __shared__ int scratch[2 * 512 + 1];
+        plan_block<256>(plan, scratch, 512);
         return;
     }
     const int d_qk = d_n + d_r;
@@ -145,13 +146,14 @@ __global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *
                                                            const int *__restrict__ seq_lens, int rows, int s_q,
                                                            int H, int hpw, float base,
                                                            __nv_bfloat16 *__restrict__ q_abs, PlanArgs plan) {
-    step_begin();
-    if (blockIdx.x == H) {   // the extra column of blocks: its first block builds the split plan
-        if (blockIdx.y == 0 && blockIdx.z == 0) plan_block<256>(plan);
-        return;
-    }
+    step_allow_next();   // loads and products touch inputs only; every store waits (below)
     __shared__ __align__(16) __nv_bfloat16 As[AB_M * AB_LD];    // [64 rows][128 k]
     __shared__ __align__(16) __nv_bfloat16 Bs[AB_K * AB_LDB];   // [128 k][64 n]
+    if (blockIdx.x == H) {   // the extra column of blocks: its first block builds the split plan
+        constexpr int CAP = ((int)sizeof(As) / 4 - 1) / 2;      // row starts and lengths in As
+        if (blockIdx.y == 0 && blockIdx.z == 0) plan_block<256>(plan, reinterpret_cast<int *>(As), CAP);
+        return;
+    }
     const int h = blockIdx.x, n0 = blockIdx.y * AB_N, row0 = blockIdx.z * AB_M;
     const int w = h / hpw, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     constexpr int D_C = 512, D_N = 128, D_R = 64, D_QK = 192, D_OUT = 576;
@@ -192,6 +194,7 @@ __global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *
         }
     }
     const int gid = lane / 4, t4 = lane % 4;
+    step_wait_prev();   // q_abs is workspace the previous call's kernels may still read
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
         const int row = row0 + wm * 16 + gid + 8 * hr;

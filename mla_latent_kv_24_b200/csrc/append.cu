@@ -136,7 +136,7 @@ __global__ void __cluster_dims__(AP_SPLIT, 1, 1) __launch_bounds__(256)
                       const __nv_bfloat16 *__restrict__ W_kr, const int *__restrict__ req,
                       const int *__restrict__ pos, int n_tok, const int *__restrict__ page_table, int batch,
                       int max_pages, int n_pages, float base, __nv_bfloat16 *__restrict__ cache, int *err) {
-    step_begin();
+    step_allow_next();   // loads and products touch inputs only; the cache stores wait (below)
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     constexpr int D_C = 512, D_R = 64, D_ROW = 576;
@@ -182,6 +182,7 @@ __global__ void __cluster_dims__(AP_SPLIT, 1, 1) __launch_bounds__(256)
     pq[(gid + 8) * AP_COLS + 8 * wc + 2 * t4 + 1] = acc[3];
     cluster.sync();
     if (rank == 0) {
+        step_wait_prev();
         for (int pi = tid; pi < AP_TOK * AP_COLS / 2; pi += 256) {
             const int r = pi / (AP_COLS / 2), cp = pi % (AP_COLS / 2);
             const int n = t0 + r, col = c0 + 2 * cp;

@@ -199,7 +199,7 @@ __global__ void __cluster_dims__(XS, 1, 1) __launch_bounds__(256, 4)
     combine_split_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
                          const int *__restrict__ row_first, int rows, int H, const __nv_bfloat16 *__restrict__ W_uv,
                          int hpw, __nv_bfloat16 *__restrict__ out) {
-    step_begin();
+    step_allow_next();   // the W_UV slice (an input) streams in while the decode finishes
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
     extern __shared__ __align__(16) uint8_t xsm[];
@@ -215,6 +215,7 @@ __global__ void __cluster_dims__(XS, 1, 1) __launch_bounds__(256, 4)
         cp_async16(Ws + v * X_LD + k, W + (size_t)v * CK + c0 + k, true);
     }
     cp_async_commit();
+    step_wait_prev();   // partials and row starts come from the decode
     // Merge: four rows per pass, two warps per row, each lane two adjacent columns of the slice.
     for (int r = warp / 2; r < CM; r += 4) {
         const int col = 64 * (warp % 2) + 2 * lane;              // column inside the slice
@@ -222,35 +223,47 @@ __global__ void __cluster_dims__(XS, 1, 1) __launch_bounds__(256, 4)
         if (r < nr) {
             const int row = row0 + r;
             const int k0 = row_first[row], k1 = row_first[row + 1];
-            float M = -INFINITY;
-            for (int k = k0 + lane; k < k1; k += 32) M = fmaxf(M, part_ml[((size_t)k * H + h) * 2]);
-#pragma unroll
-            for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-            float den = 0.f;
-            // Loads are issued in batches of KB before any is used: one memory latency per batch.
-            constexpr int KB = 8;
+            // One batch of up to KB chunks per memory round trip: lane u fetches chunk kb + u's
+            // (m, l), every lane its two columns of each chunk, all before any is used; the
+            // running max, sum and accumulator are rescaled between batches (exact).
+            constexpr int KB = 12;   // the largest batch that fits 64 registers (4 CTAs per SM)
+            float M = -INFINITY, den = 0.f;
             for (int kb = k0; kb < k1; kb += KB) {
-                float2 v[KB], ml[KB];
+                const int n = min(KB, k1 - kb);
+                float2 ml = make_float2(-INFINITY, 0.f);
+                if (lane < n) ml = *reinterpret_cast<const float2 *>(part_ml + ((size_t)(kb + lane) * H + h) * 2);
+                float2 v[KB];
 #pragma unroll
                 for (int u = 0; u < KB; ++u) {
-                    const int k = kb + u;
                     v[u] = make_float2(0.f, 0.f);
-                    ml[u] = make_float2(-INFINITY, 0.f);
-                    if (k < k1) {
-                        ml[u] = *reinterpret_cast<const float2 *>(part_ml + ((size_t)k * H + h) * 2);
-                        const int c = c0 + col;
+                    if (u < n) {
+                        const int k = kb + u, c = c0 + col;
                         const size_t off = OCT ? (((size_t)k * 64 + c / 8) * H + h) * 8 + c % 8
                                                : ((size_t)k * H + h) * CK + c;
                         v[u] = *reinterpret_cast<const float2 *>(part_o + off);
                     }
                 }
+                float mb = ml.x;
+#pragma unroll
+                for (int o = 16; o; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+                const float Mn = fmaxf(M, mb);
+                if (Mn == -INFINITY) continue;   // every chunk so far is empty
+                const float keep = M == -INFINITY ? 0.f : expf(M - Mn);
+                acc.x *= keep;
+                acc.y *= keep;
+                den *= keep;
+                const float wl = ml.x == -INFINITY ? 0.f : expf(ml.x - Mn);   // weight of chunk kb + lane
+                float dl = wl * ml.y;
+#pragma unroll
+                for (int o = 16; o; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+                den += dl;
 #pragma unroll
                 for (int u = 0; u < KB; ++u) {
-                    const float wk = ml[u].x == -INFINITY ? 0.f : expf(ml[u].x - M);
-                    den += wk * ml[u].y;
+                    const float wk = __shfl_sync(0xffffffffu, wl, u);
                     acc.x += wk * v[u].x;
                     acc.y += wk * v[u].y;
                 }
+                M = Mn;
             }
             const float inv = den > 0.f ? 1.f / den : 0.f;
             acc.x *= inv;

@@ -8,9 +8,12 @@ namespace {
 
 constexpr int PT = 1024;
 
+constexpr int CAP = 2048;
+
 __global__ void __launch_bounds__(PT) plan_kernel(PlanArgs a) {
     step_begin();
-    plan_block<PT>(a);
+    __shared__ int scratch[2 * CAP + 1];
+    plan_block<PT>(a, scratch, CAP);
 }
 
 }  // namespace

@@ -13,13 +13,19 @@
 
 namespace mla {
 
+// `scratch` is shared memory of the calling block (2 * cap_rows + 1 ints, the block's own
+// buffers, which the plan block does not otherwise use): batches of at most cap_rows rows keep
+// the row starts and lengths there, so the block's dependent reads (the binary searches of the
+// items) never wait on global memory.  Larger batches read them back from global memory.
 // Run by all PT threads of one block (PT a multiple of 32, at most 1024).
 template <int PT>
-__device__ __forceinline__ void plan_block(const PlanArgs &a) {
+__device__ __forceinline__ void plan_block(const PlanArgs &a, int *scratch, int cap_rows) {
     static_assert(PT % 32 == 0 && PT <= 1024, "one warp scans the warp totals");
     __shared__ int warp_sum[PT / 32];
     __shared__ int bad;
     const int rows = a.batch * a.s_q;
+    const bool in_smem = rows <= cap_rows;
+    int *s_first = scratch, *s_len = scratch + cap_rows + 1;
     const int per = ceil_div(rows, PT);
     const int r0 = min(rows, (int)threadIdx.x * per), r1 = min(rows, r0 + per);
     const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
@@ -31,6 +37,7 @@ __device__ __forceinline__ void plan_block(const PlanArgs &a) {
         const int L = a.seq_lens[b];
         if (L < a.s_q || L > a.max_pages * a.page) atomicOr(&bad, 1);
         const int len = L - a.s_q + j + 1;
+        if (in_smem) s_len[r] = len;
         local += len > 0 ? ceil_div(len, a.chunk) : 0;
     }
     // Exclusive prefix of the per-thread counts: warp scans, then a scan of the warp totals.
@@ -55,6 +62,7 @@ __device__ __forceinline__ void plan_block(const PlanArgs &a) {
     }
     __syncthreads();
     const int first = warp_sum[warp] + incl - local;
+    step_wait_prev();   // a no-op once the kernel waited; else the plan is workspace the previous call may still read
     if (bad) {
         if (threadIdx.x == 0) report(a.err, MLA_ERR_INVALID_ARG);
         for (int i = threadIdx.x; i < a.n_expected; i += PT) a.items[i] = WorkItem{0, 0, 0, 0};
@@ -65,21 +73,26 @@ __device__ __forceinline__ void plan_block(const PlanArgs &a) {
     for (int r = r0; r < r1; ++r) {
         const int b = r / a.s_q, j = r % a.s_q;
         a.row_first[r] = k;
-        k += ceil_div(a.seq_lens[b] - a.s_q + j + 1, a.chunk);
+        if (in_smem) s_first[r] = k;
+        k += ceil_div(in_smem ? s_len[r] : a.seq_lens[b] - a.s_q + j + 1, a.chunk);
     }
-    if (threadIdx.x == PT - 1) a.row_first[rows] = a.n_expected;
-    __syncthreads();   // row_first (global) is visible to the whole block after this barrier
+    if (threadIdx.x == PT - 1) {
+        a.row_first[rows] = a.n_expected;
+        if (in_smem) s_first[rows] = a.n_expected;
+    }
+    __syncthreads();   // row_first (shared and global) is visible to the whole block after this barrier
+    const int *rf = in_smem ? s_first : a.row_first;
     // Items in parallel: item i belongs to the last row r with row_first[r] <= i.
     for (int i = threadIdx.x; i < a.n_expected; i += PT) {
         int lo = 0, hi = rows - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) / 2;
-            if (a.row_first[mid] <= i) lo = mid;
+            if (rf[mid] <= i) lo = mid;
             else hi = mid - 1;
         }
         const int b = lo / a.s_q, j = lo % a.s_q;
-        const int len = a.seq_lens[b] - a.s_q + j + 1;
-        const int c = i - a.row_first[lo];
+        const int len = in_smem ? s_len[lo] : a.seq_lens[b] - a.s_q + j + 1;
+        const int c = i - rf[lo];
         a.items[i] = WorkItem{lo, c * a.chunk, min(len, (c + 1) * a.chunk), c};
     }
 }
