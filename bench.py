@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work budget of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads' kernel and step timings (reported under `secondary`)")
+    ap.add_argument("--secondary-steps", type=int, default=20)
     a = ap.parse_args()
     if a.warmup < 3:
         a.warmup = 3
@@ -226,6 +229,128 @@ def reduce_over_ranks(dist, device, times_ms, tokens):
     return t.tolist(), n.item()
 
 
+# --------------------------------------------------------------------------- secondary workloads
+# Workloads timed beside the headline one, each on its own path: the absorbed path on the short
+# uniform and the ragged MTP batches, the grouped (GQA) path on the GQLA batches at 8K (s_q 1, 2)
+# and 64K (s_q 2) tokens.
+SECONDARY = [("2", "absorbed"), ("4", "absorbed"), ("5_8192_1", "grouped"), ("5_8192_2", "grouped"),
+             ("5_65536_2", "grouped")]
+
+
+def device_inputs(w, seed, dev):
+    """Seeded inputs of workload `w` drawn on the device (torch Philox), with the recipe's shapes and
+    distributions (std 0.02 weights, std 1 latents / queries / hidden states, bf16), and the
+    recipe's host-side lengths and page table.  Used for the secondary timings, whose multi-GB
+    caches would take a minute to draw on the host; parity is tested on the host-drawn inputs."""
+    import torch
+    rng = np.random.default_rng(seed)
+    lens = wl.seq_lens(w, rng)
+    pt, n_pages = wl.page_table(w, lens, rng)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    def normal(shape, std):
+        return (torch.randn(shape, generator=g, device=dev, dtype=torch.float32) * std).to(torch.bfloat16)
+    t = {"W_uk": normal((w.n_w, w.d_n, w.d_c), 0.02), "W_uv": normal((w.n_w, w.d_v, w.d_c), 0.02),
+         "W_dkv": normal((w.d_c, w.hidden), 0.02), "W_kr": normal((w.d_r, w.hidden), 0.02),
+         "q": normal((w.B, w.s_q, w.H, w.d_qk), 1.0), "h": normal((w.B * w.s_q, w.hidden), 1.0)}
+    cache = torch.empty((n_pages, w.page, w.d_row), dtype=torch.bfloat16, device=dev)
+    for p0 in range(0, n_pages, 4096):
+        p1 = min(n_pages, p0 + 4096)
+        cache[p0:p1] = normal((p1 - p0, w.page, w.d_row), 1.0)
+    t["cache"] = cache
+    return lens, pt, n_pages, t
+
+
+def time_secondary(key, path, steps, warmup, dev, peaks):
+    """Kernel and step time of one secondary workload (inputs resident in HBM, L2 flushed between
+    steps when the step's bytes fit in twice the L2), with the clocks seen meanwhile."""
+    import torch
+    import mla_latent_kv_24_b200 as mla
+    w = wl.WORKLOADS[key]
+    lens, pt_np, n_pages, t = device_inputs(w, w.seed + 7919, dev)
+    dims = mla.make_dims(n_heads=w.H, heads_per_group=w.hpw, d_c=w.d_c, d_rope=w.d_r, d_nope=w.d_n, d_v=w.d_v,
+                         page_size=w.page, softmax_scale=w.softmax_scale, rope_base=w.rope_base, dtype=w.dtype)
+    page_table = torch.from_numpy(pt_np).to(dev)
+    seq_lens = torch.from_numpy(lens).to(dev)
+    req_np, pos_np = wl.new_token_positions(lens, w.s_q)
+    req, pos = torch.from_numpy(req_np).to(dev), torch.from_numpy(pos_np).to(dev)
+    max_pages = pt_np.shape[1]
+    out = torch.empty((w.B, w.s_q, w.H, w.d_v), dtype=torch.bfloat16, device=dev)
+    grouped = path == "grouped"
+    if grouped:
+        expanded = torch.empty((n_pages, w.n_w, w.page, w.d_n + w.d_v), dtype=torch.bfloat16, device=dev)
+        mla.gqla_expand_cache(dims, t["W_uk"], t["W_uv"], t["cache"], None, 0, n_pages, expanded)
+        nb = mla.gqla_decode_workspace_size(dims, w.B, w.s_q, lens)
+    else:
+        nb = mla.mla_decode_workspace_size(dims, w.B, w.s_q, lens)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=dev)
+    acct = algorithmic(w, lens, path)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if acct["step_bytes"] < 2 * L2_BYTES else None
+
+    def step():
+        mla.mla_cache_append(dims, t["h"], w.hidden, t["W_dkv"], t["W_kr"], req, pos, len(req_np), page_table, w.B,
+                             max_pages, n_pages, t["cache"])
+        if grouped:
+            mla.gqla_expand_tokens(dims, t["W_uk"], t["W_uv"], t["cache"], req, pos, len(req_np), page_table, w.B,
+                                   max_pages, n_pages, expanded)
+            mla.gqla_decode_grouped(dims, t["q"], expanded, t["cache"], page_table, seq_lens, lens, w.B, w.s_q,
+                                    max_pages, n_pages, out, ws)
+        else:
+            mla.mla_decode_absorbed(dims, t["q"], t["W_uk"], t["W_uv"], t["cache"], page_table, seq_lens, lens, w.B,
+                                    w.s_q, max_pages, n_pages, out, ws)
+
+    for _ in range(warmup):
+        step()
+    mla.mla_get_device_status()
+    # enough steps for the clock sampler (50 ms period) to see the timed region several times
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record()
+    for _ in range(3):
+        step()
+    c1.record()
+    torch.cuda.synchronize()
+    per_step_s = max(c0.elapsed_time(c1) / 3e3, 1e-6)
+    steps = int(min(4000, max(steps, 0.4 / per_step_s)))
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(4)) for _ in range(steps)]
+    for e in ev:
+        for x in e:
+            x.record()
+    torch.cuda.synchronize()
+    clocks = Clocks(dev.index or 0)
+    clocks.start()
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        s0, s1, k0, k1 = ev[i]
+        mla.mla_set_profile_events(k0, k1)
+        s0.record()
+        step()
+        s1.record()
+    mla.mla_set_profile_events(None, None)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    mla.mla_get_device_status()
+    step_us = statistics.mean(s0.elapsed_time(s1) for s0, s1, _, _ in ev) * 1e3
+    kern_us = statistics.mean(k0.elapsed_time(k1) for _, _, k0, k1 in ev) * 1e3
+    kb, kf = acct["kernel_bytes"], acct["kernel_flops"]
+    t_hbm = kb / (peaks["hbm_gbs"] * 1e9)
+    t_tc = kf / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if (t_hbm >= t_tc or grouped) else "tensor"
+    ks = kern_us / 1e6
+    achieved = kb / ks / 1e9 if bound == "hbm" else kf / ks / 1e12
+    peak = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"]
+    res = {"workload": w.name, "path": path, "kernel_us": kern_us, "step_us": step_us, "bound": bound,
+           "achieved": achieved, "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": achieved / peak,
+           "kernel_tbs": kb / ks / 1e12, "kernel_tflops": kf / ks / 1e12,
+           "cache_tokens_per_s": acct["tokens"] / (step_us / 1e6), "steps": steps, "clocks": clk,
+           "inputs": "device-drawn (seeded)"}
+    del t, ws, out
+    if grouped:
+        del expanded
+    torch.cuda.empty_cache()
+    return res
+
+
 # --------------------------------------------------------------------------- GPU arm
 def run_ours(a, rank, world, local_rank):
     import torch
@@ -382,10 +507,14 @@ def run_ours(a, rank, world, local_rank):
         if e2e is not None:
             line["e2e"] = {"value": tokens_all * a.steps / (e2e_ms / 1e3), "unit": UNIT,
                            "h2d_bytes_per_step": e2e[1], "d2h_bytes_per_step": e2e[2]}
+        if world == 1 and not a.no_secondary:
+            line["secondary"] = [time_secondary(k, pth, a.secondary_steps, a.warmup, dev, peaks)
+                                 for k, pth in SECONDARY if k != a.workload]
         if world == 1 and not a.no_cpu_baseline:
             est, units, spent, desc = oracle_sample(inp, a.cpu_seconds)
             line["cpu_baseline"] = {"value": acct["tokens"] / est, "unit": UNIT, "cores": blas_threads(),
-                                    "kind": "oracle", "sample": desc, "seconds": spent}
+                                    "kind": "oracle", "sample": desc, "seconds": spent,
+                                    "estimated": True}
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -409,12 +538,15 @@ def run_reference(a, rank, world):
     est = statistics.mean(ests)
     value = acct["tokens"] / est
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
-            "ms_per_step": est * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": est * 1e3, "ms_per_step_kind": "estimated: the oracle timed on a sample of "
+            "(request, weight-group) units, scaled by length to the whole workload",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic: seeded normal latents/queries, N(0,0.02) weights, rounded to bf16",
             "config": {"workload": w.name, "path": a.path, "batch_per_gpu": w.B, "s_q": w.s_q,
                        "cache_len": "ragged" if w.lens is None else int(w.lens[0]), "tokens_per_gpu": acct["tokens"]},
             "impl": "reference",
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc,
+                             "estimated": True},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
