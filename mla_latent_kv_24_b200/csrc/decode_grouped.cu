@@ -19,9 +19,9 @@
 // the group's 8 heads): every K/V fragment a warp loads from shared memory feeds both tiles, so
 // the four queries still share each page read from HBM.
 //
-// The head-expanded prefill ("GQLA ..." abstract: MLA's absorbed and head-expanded forms) has
-// its own kernel below: one CTA per (head, 64-query tile), each warp owning 16 queries over all
-// tokens of the tile's causal range.
+// The head-expanded prefill ("GQLA ..." abstract: MLA's absorbed and head-expanded forms) is
+// compute-dense and runs on the 5th-generation tensor cores (prefill_tc.cu); only its launcher
+// lives here, beside the grouped decode whose cache it reads.
 #include <math.h>
 
 #include "tc_decode.h"
@@ -321,182 +321,6 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
 }
 
 
-// Head-expanded prefill: one CTA takes one head and PQ = 64 consecutive query tokens of one
-// request; warp w owns queries [16 w, 16 w + 16) of the tile over every token (the usual
-// flash-attention split), so each page of K|V and k^R is read once per 64 queries.  Pages after
-// the tile's last query position are skipped; the diagonal pages are masked per element.
-constexpr int PW = 4, PQ = 16 * PW;
-constexpr size_t P_SMEM = sizeof(__nv_bfloat16) * ((size_t)STAGES * (KV_TILE + KR_TILE) + (size_t)PQ * Q_LD);
-
-__global__ void __launch_bounds__(PW * 32, 2) prefill_kernel(GParams p) {
-    step_begin();
-    extern __shared__ __align__(16) uint8_t psm[];
-    __nv_bfloat16 *kv = reinterpret_cast<__nv_bfloat16 *>(psm);      // [STAGES][64][KV_LD]
-    __nv_bfloat16 *kr = kv + STAGES * KV_TILE;                         // [STAGES][64][KR_LD]
-    __nv_bfloat16 *qs = kr + STAGES * KR_TILE;                         // [PQ][Q_LD]
-    const int head = blockIdx.x, item = blockIdx.y, q0 = PQ * blockIdx.z;
-    if (item >= p.plan.n_work) return;
-    const WorkItem it = p.plan.items[item];
-    const int n_q = p.s_q;
-    const int g = head / p.hpw, G = p.H / p.hpw;
-    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-    const int b = it.row;
-    const int L = p.seq_lens[b];
-    const int q_last = min(n_q, q0 + PQ) - 1;
-    const int t_end = min(it.t1, L - n_q + q_last + 1);
-    const int n_pg = t_end > it.t0 ? ceil_div(t_end - it.t0, PAGE) : 0;
-    const size_t part_base = (size_t)item * n_q;
-
-    for (int i = tid; i < PQ * (D_QK / 8); i += blockDim.x) {   // 16-byte chunks of the query tile
-        const int m = i / (D_QK / 8), c = 8 * (i % (D_QK / 8)), q = q0 + m;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (q < n_q) v = *reinterpret_cast<const uint4 *>(p.q + (((size_t)b * n_q + q) * p.H + head) * D_QK + c);
-        *reinterpret_cast<uint4 *>(qs + m * Q_LD + c) = v;
-    }
-    auto load_page = [&](int stage, int i) {
-        int pid = p.page_table[(size_t)b * p.max_pages + it.t0 / PAGE + i];
-        bool ok = true;
-        if (pid < 0 || pid >= p.n_pages) {
-            if (tid == 0) report(p.err, MLA_ERR_DEVICE_BOUNDS);
-            ok = false;
-            pid = 0;
-        }
-        const int valid = ok ? min(PAGE, it.t1 - (it.t0 + PAGE * i)) : 0;
-        const __nv_bfloat16 *src_kv = p.expanded + (((size_t)pid * G + g) * PAGE) * 256;
-        const __nv_bfloat16 *src_kr = p.latent + ((size_t)pid * PAGE) * D_ROW + D_LAT;
-        __nv_bfloat16 *dkv = kv + stage * KV_TILE, *dkr = kr + stage * KR_TILE;
-        for (int c = tid; c < PAGE * 32; c += blockDim.x) {
-            const int r = c / 32, k = (c % 32) * 8;
-            cp_async16(dkv + r * KV_LD + k, src_kv + (size_t)r * 256 + k, r < valid);
-        }
-        for (int c = tid; c < PAGE * 8; c += blockDim.x) {
-            const int r = c / 8, k = (c % 8) * 8;
-            cp_async16(dkr + r * KR_LD + k, src_kr + (size_t)r * D_ROW + k, r < valid);
-        }
-    };
-    if (n_pg > 0) load_page(0, 0);
-    cp_async_commit();
-    __syncthreads();   // the query tile is in shared memory
-
-    uint32_t qa[12][4];
-#pragma unroll
-    for (int ks = 0; ks < 12; ++ks)
-        ldmatrix_x4(qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3],
-                    qs + (16 * warp + (lane % 8) + 8 * ((lane / 8) % 2)) * Q_LD + 16 * ks + 8 * (lane / 16));
-
-    const int gid = lane / 4, t4 = lane % 4;
-    const int qa0 = q0 + 16 * warp + gid, qa1 = qa0 + 8;          // this thread's two query rows
-    const int lim0 = qa0 < n_q ? L - n_q + qa0 : -1;              // last visible token of each
-    const int lim1 = qa1 < n_q ? L - n_q + qa1 : -1;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float o[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-
-    for (int i = 0; i < n_pg; ++i) {
-        if (i + 1 < n_pg) load_page((i + 1) % STAGES, i + 1);
-        cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
-        const __nv_bfloat16 *tkv = kv + (i % STAGES) * KV_TILE;
-        const __nv_bfloat16 *tkr = kr + (i % STAGES) * KR_TILE;
-        // S [16 rows x 64 tokens] = Q~ K~^T over 192 dims.
-        float s[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 12; ks += 2) {
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                uint32_t bf[4];
-                const int tok = 8 * nt + (lane % 8);
-                const __nv_bfloat16 *src = ks < 8 ? tkv + tok * KV_LD + 16 * ks + 8 * (lane / 8)
-                                                  : tkr + tok * KR_LD + 16 * (ks - 8) + 8 * (lane / 8);
-                ldmatrix_x4(bf[0], bf[1], bf[2], bf[3], src);
-                mma_bf16(s[nt], qa[ks], bf[0], bf[1]);
-                mma_bf16(s[nt], qa[ks + 1], bf[2], bf[3]);
-            }
-        }
-        const int tok_base = it.t0 + PAGE * i;
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int t = tok_base + 8 * nt + 2 * t4 + e;
-                const bool in = t < it.t1;
-                s[nt][e] = (in && t <= lim0) ? s[nt][e] * p.scale_log2 : -INFINITY;
-                s[nt][2 + e] = (in && t <= lim1) ? s[nt][2 + e] * p.scale_log2 : -INFINITY;
-                mx0 = fmaxf(mx0, s[nt][e]);
-                mx1 = fmaxf(mx1, s[nt][2 + e]);
-            }
-#pragma unroll
-        for (int off = 1; off <= 2; off <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-        }
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-        const float a0 = n0 == -INFINITY ? 1.f : exp2f(m0 - n0), a1 = n1 == -INFINITY ? 1.f : exp2f(m1 - n1);
-        float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                s[nt][e] = n0 == -INFINITY ? 0.f : exp2f(s[nt][e] - n0);
-                s[nt][2 + e] = n1 == -INFINITY ? 0.f : exp2f(s[nt][2 + e] - n1);
-                sum0 += s[nt][e];
-                sum1 += s[nt][2 + e];
-            }
-        l0 = l0 * a0 + sum0;
-        l1 = l1 * a1 + sum1;
-        m0 = n0;
-        m1 = n1;
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            o[n][0] *= a0;
-            o[n][1] *= a0;
-            o[n][2] *= a1;
-            o[n][3] *= a1;
-        }
-        // O [16 x 128] += P V, 16 tokens per k-step; P's accumulator layout is the A fragment.
-#pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-            const uint32_t pa[4] = {pack_bf16(s[2 * kt][0], s[2 * kt][1]), pack_bf16(s[2 * kt][2], s[2 * kt][3]),
-                                    pack_bf16(s[2 * kt + 1][0], s[2 * kt + 1][1]),
-                                    pack_bf16(s[2 * kt + 1][2], s[2 * kt + 1][3])};
-#pragma unroll
-            for (int n = 0; n < 16; n += 2) {
-                uint32_t vb[4];
-                const __nv_bfloat16 *src =
-                    tkv + (16 * kt + (lane % 8) + 8 * ((lane / 8) % 2)) * KV_LD + D_N + 8 * n + 8 * (lane / 16);
-                ldmatrix_x4_trans(vb[0], vb[1], vb[2], vb[3], src);
-                mma_bf16(o[n], pa, vb[0], vb[1]);
-                mma_bf16(o[n + 1], pa, vb[2], vb[3]);
-            }
-        }
-        __syncthreads();   // this stage is refilled by the next iteration's load
-    }
-    cp_async_wait<0>();
-#pragma unroll
-    for (int off = 1; off <= 2; off <<= 1) {
-        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-    }
-    // Each warp owns its rows: write the partial (relative to m, log2 units) and (m, l) directly.
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-        const int q = hr ? qa1 : qa0;
-        if (q >= n_q) continue;
-        const size_t r = (part_base + q) * p.H + head;
-#pragma unroll
-        for (int n = 0; n < 16; ++n)
-            *reinterpret_cast<float2 *>(p.part_o + r * D_V + 8 * n + 2 * t4) = make_float2(o[n][2 * hr], o[n][2 * hr + 1]);
-        if (t4 == 0) {
-            p.part_ml[r * 2] = (hr ? m1 : m0) * 0.69314718055994531f;
-            p.part_ml[r * 2 + 1] = hr ? l1 : l0;
-        }
-    }
-}
 }  // namespace
 
 bool grouped_tc_ok(const Dims &d, int s_q) {
@@ -554,15 +378,8 @@ bool prefill_ok(const Dims &d) {
 cudaError_t launch_prefill_expanded(const Dims &d, const void *q_rot, const void *expanded, const void *latent,
                                     const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
                                     int n_pages, int n_q, float *part_o, float *part_ml, int *err, cudaStream_t st) {
-    if (plan.n_work == 0) return cudaSuccess;
-    if (plan.n_work > 65535 || ceil_div(n_q, PQ) > 65535) return cudaErrorInvalidValue;
-    const GParams p = grouped_params(d, q_rot, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages, n_q,
-                                     part_o, part_ml, err);
-    cudaError_t e = raise_smem_limit((const void *)prefill_kernel, P_SMEM);
-    if (e != cudaSuccess) return e;
-    dim3 grid(d.H, plan.n_work, ceil_div(n_q, PQ));
-    MLA_STEP_LAUNCH(prefill_kernel, dim3(grid), dim3(PW * 32), P_SMEM, st, p);
-    return cudaGetLastError();
+    return launch_prefill_tc(d, q_rot, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages, n_q, part_o,
+                             part_ml, err, st);
 }
 
 }  // namespace mla

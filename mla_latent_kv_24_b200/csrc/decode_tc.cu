@@ -131,7 +131,7 @@ __device__ __forceinline__ bool wait_or_abort(const Ctx &c, uint32_t bar, uint32
     return false;
 }
 
-// Same, with one verdict for the whole warp (the tcgen05 loads that follow are warp-collective).
+// Same, with one answer for the whole warp (the tcgen05 loads that follow are warp-collective).
 __device__ __forceinline__ bool warp_wait(const Ctx &c, uint32_t bar, uint32_t parity, int *err) {
     const bool ok = wait_or_abort(c, bar, parity, err);
     return __all_sync(0xffffffffu, ok);

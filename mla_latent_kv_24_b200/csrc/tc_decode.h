@@ -30,6 +30,10 @@ bool prefill_ok(const Dims &d);
 cudaError_t launch_prefill_expanded(const Dims &d, const void *q_rot, const void *expanded, const void *latent,
                                     const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
                                     int n_pages, int n_q, float *part_o, float *part_ml, int *err, cudaStream_t st);
+// tcgen05 head-expanded prefill (prefill_tc.cu), the kernel behind launch_prefill_expanded.
+cudaError_t launch_prefill_tc(const Dims &d, const void *q_rot, const void *expanded, const void *latent,
+                              const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
+                              int n_pages, int n_q, float *part_o, float *part_ml, int *err, cudaStream_t st);
 cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expanded, const void *latent,
                                   const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
                                   int n_pages, int s_q, float *part_o, float *part_ml, int *err, cudaStream_t st);

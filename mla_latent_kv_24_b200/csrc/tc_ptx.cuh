@@ -147,9 +147,9 @@ __device__ __forceinline__ void mma_pair_bf16_k(uint32_t d_tmem, uint64_t a_desc
                      "r"(idesc)
                      : "memory");
 }
-// Same with A read from tensor memory: each CTA's A rows at `a_tmem` in the layout the two-CTA
-// form takes for M = 128, the CTA's 64 rows in lanes 0-63 and again in lanes 64-127 (K pairs of
-// bf16 packed per 32-bit column).
+// Same with A read from tensor memory at `a_tmem` in each CTA, K pairs of bf16 packed per 32-bit
+// column.  With M = 256 each CTA's 128 rows take one lane each; with M = 128 the two-CTA form
+// takes the CTA's 64 rows in lanes 0-63 and again in lanes 64-127.
 template <bool ACCUMULATE>
 __device__ __forceinline__ void mma_pair_ts_bf16_k(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc) {
     if (ACCUMULATE)
