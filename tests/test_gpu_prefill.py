@@ -41,3 +41,15 @@ def test_full_prefill_from_an_empty_context():
     assert_close(got, ref, "bf16", "full prefill")
     # query 0 sees only token 0, so each head's output is its V row of token 0 (one-key softmax)
     np.testing.assert_allclose(got[0, 0], ref[0, 0], rtol=0, atol=2 ** -7 * np.abs(ref[0, 0]).max())
+
+
+def test_prefill_full_size_sampled():
+    # the size the prefill is timed at: B = 2, L = 4096, n_q = 512 (per-head cache), sampled rows
+    from _gpu import compare_sampled, oracle_decode_sampled, sample_outputs
+    w = wl.small_workload(wl.WORKLOADS["2"], B=2, s_q=512, lens=[4096, 4096], seed=7)
+    inp = wl.make_inputs(w)
+    dev = Dev(inp)
+    got = wl.from_torch_f64(prefill(dev, dev.expand()))
+    assert np.isfinite(got).all()
+    sample = sample_outputs(inp, 24)
+    compare_sampled(got, oracle_decode_sampled(inp, sample), "bf16", "prefill B=2 L=4096 n_q=512")
