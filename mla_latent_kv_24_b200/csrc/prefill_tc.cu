@@ -13,7 +13,9 @@
 //                (K_g from the expanded cache, k^R from the latent cache).
 //   O += P V     M=256, N=128 (d_v), K=128 tokens: P is read from TMEM (each CTA's 128 rows, one
 //                lane per query), CTA r supplies d_v columns [64 r, +64) of both pages.
-// TMEM per CTA: two S buffers (128 columns each), O (128), P (64 columns of bf16 pairs).
+// TMEM per CTA: two S buffers (128 columns each), O (128) and two P buffers (64 columns of bf16
+// pairs each), so the softmax of step i waits for PV(i-2) before writing P, and for PV(i-1) only
+// when it rescales O.
 // Shared memory: Q (128 queries x 192, 48 KiB), a K ring (one page per slot: 16 KiB of K_g and
 // 8 KiB of k^R) and a V ring (one step per slot: 2 pages x 64 d_v columns, 16 KiB).
 // Warp roles (256 threads): warps 0-3 softmax (thread = query row) and epilogue, warp 4 K/Q
@@ -51,7 +53,7 @@ enum {
     B_SFULL,
     B_SFREE = B_SFULL + 2,
     B_PFULL = B_SFREE + 2,
-    B_PVDONE,
+    B_PVDONE = B_PFULL + 2,
     B_COUNT = B_PVDONE + 2
 };
 constexpr uint32_t OFF_TMEMPTR = OFF_BAR + B_COUNT * 8;
@@ -62,7 +64,7 @@ static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 constexpr uint32_t TM_S = 0;      // two S buffers of 128 columns
 constexpr uint32_t TM_O = 256;    // O: 128 columns
-constexpr uint32_t TM_P = 384;    // P: 64 columns of bf16 pairs
+constexpr uint32_t TM_P = 384;    // P: two buffers of 64 columns of bf16 pairs
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(256, 128, false, false);
@@ -212,12 +214,12 @@ __device__ void run_pv_issuer(const Ctx &c, const PfParams &p, const Unit &u, ui
     const uint64_t vdesc = tc::sdesc_sw128(c.base + OFF_V, KBLK, 1024);
     for (int i = 0; i < u.n_steps; ++i) {
         const int slot = i % NV;
-        if (!wait_or_abort(c, c.bar(B_PFULL), (uint32_t)i & 1u, p.err)) return;
+        if (!wait_or_abort(c, c.bar(B_PFULL + (i & 1)), (uint32_t)(i >> 1) & 1u, p.err)) return;
         if (!wait_or_abort(c, c.bar(B_VFULL + slot), (uint32_t)(i / NV) & 1u, p.err)) return;
         tc::fence_after_sync();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {   // 16 tokens per instruction: page k / 4, rows 16 (k % 4)
-            const uint32_t a = tmem + TM_P + 8 * k;
+            const uint32_t a = tmem + TM_P + 64 * (i & 1) + 8 * k;
             const uint64_t b = tc::sdesc_add(vdesc, slot * VSLOT + (k / 4) * KBLK + 2048 * (k % 4));
             if (i == 0 && k == 0)
                 tc::mma_pair_ts_bf16_k<false>(tmem + TM_O, a, b, IDESC_PV);
@@ -261,7 +263,11 @@ __device__ void run_softmax(const Ctx &c, const PfParams &p, const Unit &u, uint
         }
         const bool any = __any_sync(0xffffffffu, i > 0 && mx > m_run + RESCALE_LOG2);
         // PV(i-1) must be complete before O is rescaled and before P is overwritten.
-        if (i >= 1) warp_wait(c, c.bar(B_PVDONE + ((i - 1) & 1)), (uint32_t)((i - 1) >> 1) & 1u, p.err);
+        // P is double-buffered: P(i) needs PV(i-2) complete; a rescale of O needs PV(i-1).
+        if (any && i >= 1)
+            warp_wait(c, c.bar(B_PVDONE + ((i - 1) & 1)), (uint32_t)((i - 1) >> 1) & 1u, p.err);
+        else if (i >= 2)
+            warp_wait(c, c.bar(B_PVDONE + (i & 1)), (uint32_t)((i - 2) >> 1) & 1u, p.err);
         tc::fence_after_sync();
         if (i == 0) {
             m_run = mx;
@@ -292,11 +298,11 @@ __device__ void run_softmax(const Ctx &c, const PfParams &p, const Unit &u, uint
             pk[j] = *reinterpret_cast<uint32_t *>(&h2);
         }
         l_run += sum;
-        tc::tmem_st64(tmem + TM_P + lane_addr, reinterpret_cast<const float *>(pk));
+        tc::tmem_st64(tmem + TM_P + 64 * (i & 1) + lane_addr, reinterpret_cast<const float *>(pk));
         tc::tmem_wait_st();
         tc::fence_before_sync();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive_cluster(c.lead_bar(B_PFULL));
+        if (lane == 0) tc::mbar_arrive_cluster(c.lead_bar(B_PFULL + (i & 1)));
     }
     // Epilogue: the unnormalised O (relative to m, log2 units), m in natural-log units, and l.
     if (u.n_steps > 0) {
@@ -362,6 +368,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             tc::mbar_init(c.bar(B_PVDONE + i), 1);
         }
         tc::mbar_init(c.bar(B_PFULL), 2 * SM_WARPS);
+        tc::mbar_init(c.bar(B_PFULL + 1), 2 * SM_WARPS);
         *c.abort_flag = 0;
         tc::fence_mbar_init();
     }
