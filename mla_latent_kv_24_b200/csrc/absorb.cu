@@ -139,30 +139,37 @@ cudaError_t launch_q_rope(const Dims &d, const void *q, const int *seq_lens, int
 namespace mla {
 namespace {
 
-constexpr int AB_M = 64, AB_N = 64, AB_K = 128, AB_LD = AB_K + 8, AB_LDB = AB_N + 8;
+constexpr int AB_K = 128, AB_LD = AB_K + 8;
 
+// TM query rows x TN latent columns of one head per CTA; eight warps as (TM / 16) row tiles x
+// (8 / (TM / 16)) column groups.  Small batches take 16 x 128 tiles, so that a decode step's
+// whole grid (4 column tiles per head) is one wave of CTAs: a CTA stores only after the previous
+// kernel has completed, and a second wave would start its loads only then.
+template <int TM, int TN>
 __global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *__restrict__ q,
                                                            const __nv_bfloat16 *__restrict__ W_uk,
                                                            const int *__restrict__ seq_lens, int rows, int s_q,
                                                            int H, int hpw, float base,
                                                            __nv_bfloat16 *__restrict__ q_abs, PlanArgs plan) {
+    constexpr int LDB = TN + 8, WM = TM / 16, WN = 8 / WM, CW = TN / WN, NT = CW / 8;
+    static_assert(TM % 16 == 0 && 8 % WM == 0 && NT % 2 == 0, "warp tiling");
     step_allow_next();   // loads and products touch inputs only; every store waits (below)
-    __shared__ __align__(16) __nv_bfloat16 As[AB_M * AB_LD];    // [64 rows][128 k]
-    __shared__ __align__(16) __nv_bfloat16 Bs[AB_K * AB_LDB];   // [128 k][64 n]
+    __shared__ __align__(16) __nv_bfloat16 As[TM * AB_LD];     // [rows][128 k]
+    __shared__ __align__(16) __nv_bfloat16 Bs[AB_K * LDB];     // [128 k][TN n]
     if (blockIdx.x == H) {   // the extra column of blocks: its first block builds the split plan
-        constexpr int CAP = ((int)sizeof(As) / 4 - 1) / 2;      // row starts and lengths in As
-        if (blockIdx.y == 0 && blockIdx.z == 0) plan_block<256>(plan, reinterpret_cast<int *>(As), CAP);
+        constexpr int CAP = ((int)sizeof(Bs) / 4 - 1) / 2;      // row starts and lengths in Bs
+        if (blockIdx.y == 0 && blockIdx.z == 0) plan_block<256>(plan, reinterpret_cast<int *>(Bs), CAP);
         return;
     }
-    const int h = blockIdx.x, n0 = blockIdx.y * AB_N, row0 = blockIdx.z * AB_M;
+    const int h = blockIdx.x, n0 = blockIdx.y * TN, row0 = blockIdx.z * TM;
     const int w = h / hpw, tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     constexpr int D_C = 512, D_N = 128, D_R = 64, D_QK = 192, D_OUT = 576;
     const __nv_bfloat16 *Wk = W_uk + (size_t)w * D_N * D_C;
-    for (int c = tid; c < AB_K * AB_N / 8; c += 256) {          // 2048 chunks of 16 B
-        const int k = c / (AB_N / 8), n = (c % (AB_N / 8)) * 8;
-        cp_async16(Bs + k * AB_LDB + n, Wk + (size_t)k * D_C + n0 + n, true);
+    for (int c = tid; c < AB_K * TN / 8; c += 256) {            // 16-byte chunks of the W_UK tile
+        const int k = c / (TN / 8), n = (c % (TN / 8)) * 8;
+        cp_async16(Bs + k * LDB + n, Wk + (size_t)k * D_C + n0 + n, true);
     }
-    for (int c = tid; c < AB_M * AB_K / 8; c += 256) {
+    for (int c = tid; c < TM * AB_K / 8; c += 256) {
         const int r = c / (AB_K / 8), k = (c % (AB_K / 8)) * 8;
         const int row = row0 + r;
         cp_async16(As + r * AB_LD + k, q + ((size_t)(row < rows ? row : 0) * H + h) * D_QK + k, row < rows);
@@ -170,11 +177,11 @@ __global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
-    // warp tile: 16 rows x 32 columns (4 n8 tiles); 4 x 2 warps cover 64 x 64
-    const int wm = warp % 4, wn = warp / 4;
-    float acc[4][4];
+    // warp tile: 16 rows x CW columns (NT n8 tiles)
+    const int wm = warp % WM, wn = warp / WM;
+    float acc[NT][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < NT; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[j][e] = 0.f;
 #pragma unroll
@@ -183,12 +190,12 @@ __global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *
         ldmatrix_x4(a[0], a[1], a[2], a[3],
                     As + (wm * 16 + (lane % 8) + 8 * ((lane / 8) % 2)) * AB_LD + kk + 8 * (lane / 16));
 #pragma unroll
-        for (int j = 0; j < 4; j += 2) {
+        for (int j = 0; j < NT; j += 2) {
             // B stored [k][n]: .trans gives the k-major fragments of two n8 tiles
             uint32_t b0, b1, b2, b3;
             const int kr = kk + (lane % 8) + 8 * ((lane / 8) % 2);
-            const int nc = wn * 32 + j * 8 + 8 * (lane / 16);
-            ldmatrix_x4_trans(b0, b1, b2, b3, Bs + kr * AB_LDB + nc);
+            const int nc = wn * CW + j * 8 + 8 * (lane / 16);
+            ldmatrix_x4_trans(b0, b1, b2, b3, Bs + kr * LDB + nc);
             mma_bf16(acc[j], a, b0, b1);
             mma_bf16(acc[j + 1], a, b2, b3);
         }
@@ -199,13 +206,13 @@ __global__ void __launch_bounds__(256) q_absorb_mma_kernel(const __nv_bfloat16 *
     for (int hr = 0; hr < 2; ++hr) {
         const int row = row0 + wm * 16 + gid + 8 * hr;
         if (row >= rows) continue;
-        __nv_bfloat16 *dst = q_abs + ((size_t)row * H + h) * D_OUT + n0 + wn * 32;
+        __nv_bfloat16 *dst = q_abs + ((size_t)row * H + h) * D_OUT + n0 + wn * CW;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < NT; ++j)
             *reinterpret_cast<uint32_t *>(dst + j * 8 + 2 * t4) = pack_bf16(acc[j][2 * hr], acc[j][2 * hr + 1]);
     }
     if (blockIdx.y == 0) {   // RoPE part of the query, rows of this tile
-        for (int i = tid; i < AB_M * (D_R / 2); i += 256) {
+        for (int i = tid; i < TM * (D_R / 2); i += 256) {
             const int r = i / (D_R / 2), pi = i % (D_R / 2), row = row0 + r;
             if (row >= rows) continue;
             const int b = row / s_q, j = row % s_q, pos = seq_lens[b] - s_q + j;
@@ -226,10 +233,17 @@ bool q_absorb_mma_ok(const Dims &d) { return d.bf16 && d.d_n == 128 && d.d_c == 
 cudaError_t launch_q_absorb_mma(const Dims &d, const void *q, const void *W_uk, const int *seq_lens, int batch,
                                 int s_q, void *q_abs, const PlanArgs &plan, cudaStream_t st) {
     const int rows = batch * s_q;
-    dim3 grid(d.H + 1, 512 / AB_N, ceil_div(rows, AB_M));   // + one column for the plan block
-    MLA_STEP_LAUNCH(q_absorb_mma_kernel, dim3(grid), dim3(256), 0, st, (const __nv_bfloat16 *)q,
-                    (const __nv_bfloat16 *)W_uk, seq_lens, rows, s_q, d.H, d.hpw, d.base, (__nv_bfloat16 *)q_abs,
-                    plan);
+    if (rows <= 16) {
+        dim3 grid(d.H + 1, 512 / 128, 1);   // + one column for the plan block
+        MLA_STEP_LAUNCH(q_absorb_mma_kernel<16, 128>, dim3(grid), dim3(256), 0, st, (const __nv_bfloat16 *)q,
+                        (const __nv_bfloat16 *)W_uk, seq_lens, rows, s_q, d.H, d.hpw, d.base, (__nv_bfloat16 *)q_abs,
+                        plan);
+    } else {
+        dim3 grid(d.H + 1, 512 / 64, ceil_div(rows, 64));
+        MLA_STEP_LAUNCH(q_absorb_mma_kernel<64, 64>, dim3(grid), dim3(256), 0, st, (const __nv_bfloat16 *)q,
+                        (const __nv_bfloat16 *)W_uk, seq_lens, rows, s_q, d.H, d.hpw, d.base, (__nv_bfloat16 *)q_abs,
+                        plan);
+    }
     return cudaGetLastError();
 }
 

@@ -349,9 +349,21 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
             SimtDecodeArgs a{qp, latent, nullptr, page_table, plan, max_pages, n_pages, s_q, 0, part_o, part_ml, err};
             MLA_CUDA(launch_decode_simt(d, a, st), "launch decode (CUDA cores)");
         }
-        if (combine_mma_ok(d, L.DV, true))
-            MLA_CUDA(launch_combine_mma(d, part_o, part_ml, row_first, L.rows, tc, W_uv, out, st),
+        if (combine_mma_ok(d, L.DV, true)) {
+            // The plan's row starts from the host lengths (the device plan is built from the same rule).
+            int starts[RowStarts::MAX + 1];
+            const int *sp = nullptr;
+            if (L.rows <= RowStarts::MAX && L.plan_sq == s_q) {
+                starts[0] = 0;
+                for (int r = 0; r < L.rows; ++r) {
+                    const int b = r / s_q, j = r % s_q;
+                    starts[r + 1] = starts[r] + ceil_div(lens_host[b] - s_q + j + 1, L.chunk);
+                }
+                if (starts[L.rows] == L.n_work) sp = starts;
+            }
+            MLA_CUDA(launch_combine_mma(d, part_o, part_ml, row_first, sp, L.rows, tc, W_uv, out, st),
                      "launch combine + W_UV (tensor cores)");
+        }
         else if (!tc)
             MLA_CUDA(launch_combine(d, part_o, part_ml, row_first, L.rows, 1, L.DV, W_uv, out, st), "launch combine");
         else

@@ -197,8 +197,8 @@ constexpr int XS = 4, XC = CK / XS, X_LD = XC + 8;        // cluster size, colum
 template <bool OCT>
 __global__ void __cluster_dims__(XS, 1, 1) __launch_bounds__(256, 4)
     combine_split_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
-                         const int *__restrict__ row_first, int rows, int H, const __nv_bfloat16 *__restrict__ W_uv,
-                         int hpw, __nv_bfloat16 *__restrict__ out) {
+                         const int *__restrict__ row_first, const RowStarts rs, int rows, int H,
+                         const __nv_bfloat16 *__restrict__ W_uv, int hpw, __nv_bfloat16 *__restrict__ out) {
     step_allow_next();   // the W_UV slice (an input) streams in while the decode finishes
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
@@ -222,7 +222,7 @@ __global__ void __cluster_dims__(XS, 1, 1) __launch_bounds__(256, 4)
         float2 acc = make_float2(0.f, 0.f);
         if (r < nr) {
             const int row = row0 + r;
-            const int k0 = row_first[row], k1 = row_first[row + 1];
+            const int k0 = rs.n ? rs.v[row] : row_first[row], k1 = rs.n ? rs.v[row + 1] : row_first[row + 1];
             // One batch of up to KB chunks per memory round trip: lane u fetches chunk kb + u's
             // (m, l), every lane its two columns of each chunk, all before any is used; the
             // running max, sum and accumulator are rescaled between batches (exact).
@@ -322,7 +322,14 @@ bool combine_mma_ok(const Dims &d, int DV, bool project) {
 }
 
 cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
-                               int rows, bool oct_layout, const void *W_uv, void *out, cudaStream_t st) {
+                               const int *rows_host, int rows, bool oct_layout, const void *W_uv, void *out,
+                               cudaStream_t st) {
+    RowStarts rs;
+    rs.n = 0;
+    if (rows_host != nullptr && rows <= RowStarts::MAX) {
+        rs.n = rows;
+        for (int r = 0; r <= rows; ++r) rs.v[r] = rows_host[r];
+    }
     const size_t smem = sizeof(__nv_bfloat16) * (size_t)(CN + CM) * X_LD;
     static_assert(sizeof(float) * CM * CN <= sizeof(__nv_bfloat16) * CN * X_LD, "Red fits over Ws");
     if (rows <= 0) return cudaSuccess;
@@ -331,7 +338,7 @@ cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *
     auto k = oct_layout ? combine_split_kernel<true> : combine_split_kernel<false>;
     cudaError_t e = raise_smem_limit((const void *)k, smem);
     if (e != cudaSuccess) return e;
-    MLA_STEP_LAUNCH(k, dim3(grid), dim3(256), smem, st, part_o, part_ml, row_first, rows, d.H,
+    MLA_STEP_LAUNCH(k, dim3(grid), dim3(256), smem, st, part_o, part_ml, row_first, rs, rows, d.H,
                     (const __nv_bfloat16 *)W_uv, d.hpw, (__nv_bfloat16 *)out);
     return cudaGetLastError();
 }

@@ -74,9 +74,18 @@ cudaError_t launch_combine(const Dims &d, const float *part_o, const float *part
 // Tensor-core combine + W_UV for bf16, d_c = 512, d_v = 128 (combine.cu).  oct_layout: the
 // partials are in the tcgen05 decode's column-octet layout [n_work, 64, H, 8] instead of
 // [n_work, H, 512].
+// rows_host: the plan's row starts computed on the host from the host lengths (rows + 1 values),
+// or nullptr; batches of at most RowStarts::MAX rows pass them by value, which saves the kernel a
+// dependent load (the device plan still validates the lengths and reports a mismatch).
+struct RowStarts {
+    static constexpr int MAX = 64;
+    int n;              // rows covered (0: read row_first from the workspace)
+    int v[MAX + 1];
+};
 bool combine_mma_ok(const Dims &d, int DV, bool project);
 cudaError_t launch_combine_mma(const Dims &d, const float *part_o, const float *part_ml, const int *row_first,
-                               int rows, bool oct_layout, const void *W_uv, void *out, cudaStream_t st);
+                               const int *rows_host, int rows, bool oct_layout, const void *W_uv, void *out,
+                               cudaStream_t st);
 
 // Per-group cache expansion (expand.cu).
 cudaError_t launch_expand(const Dims &d, const void *W_uk, const void *W_uv, const void *latent,
