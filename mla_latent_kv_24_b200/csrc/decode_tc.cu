@@ -19,10 +19,13 @@
 //                comes from tensor memory.
 // Every CTA loads only its own tiles, from its own GPU's HBM, with plain (non-multicast) TMA.
 //
-// Warp roles (384 threads per CTA): warps 0-7 softmax + epilogue (two warps per TMEM lane
-// quadrant, each taking half of a lane's columns), warp 8 producer of Q and of the K ring,
-// warp 10 producer of the V ring, warp 9 QK^T issuer (leader CTA only) and TMEM allocator,
-// warp 11 PV issuer (leader CTA only).  Shared memory holds Q
+// Warp roles (416 threads per CTA): warps 0-7 softmax + epilogue (two warps per TMEM lane
+// quadrant, each taking half of a lane's columns), warp 8 producer of Q and of K slots 0-1,
+// warp 12 producer of K slot 2, warp 10 producer of the V ring, warp 9 QK^T issuer (leader CTA
+// only) and TMEM allocator, warp 11 PV issuer (leader CTA only).  The tensor copies one thread
+// issues are processed one after another (measured: ~250 ns per copy from L2 and ~600 ns per
+// 24 KiB box from HBM under full load, whatever the ring depth), so the K ring, which streams
+// the cache from HBM, has two issuing threads.  Shared memory holds Q
 // (72 KiB), a K ring of three 24 KiB slots (one step: the CTA's page x 576 columns as three
 // groups of three 64-column blocks), a V ring of two 32 KiB slots (one per page of the step:
 // this CTA's 256 latent columns) and a 16 KiB buffer through which the softmax threads of lanes
@@ -95,8 +98,9 @@ constexpr uint64_t WAIT_NS = 2000000000ull;   // 2 s: no legitimate wait comes n
 constexpr int SOFTMAX_WARPS = 8;
 constexpr int SM_THREADS = 32 * SOFTMAX_WARPS;
 constexpr int W_KPROD = SOFTMAX_WARPS, W_MMA = SOFTMAX_WARPS + 1, W_VPROD = SOFTMAX_WARPS + 2,
-              W_PV = SOFTMAX_WARPS + 3;
-constexpr int THREADS = 32 * (SOFTMAX_WARPS + 4);
+              W_PV = SOFTMAX_WARPS + 3, W_KPROD2 = SOFTMAX_WARPS + 4;
+constexpr int K_SPLIT = 2;   // K slots [0, K_SPLIT) come from W_KPROD, the rest from W_KPROD2
+constexpr int THREADS = 32 * (SOFTMAX_WARPS + 5);
 constexpr float RESCALE_LOG2 = 8.f;           // rescale O when a row max grows by more than 2^8
 
 struct TcParams {
@@ -123,9 +127,11 @@ struct Ctx {
     __device__ uint32_t vslot(int i) const { return base + OFF_V + VSLOT * i; }
 };
 
+// `spin`: the MMA issuers wait without suspending, so they resume as soon as a phase completes.
+template <bool spin = false>
 __device__ __forceinline__ bool wait_or_abort(const Ctx &c, uint32_t bar, uint32_t parity, int *err) {
     if (*c.abort_flag) return false;
-    if (tc::mbar_wait(bar, parity, c.wait_ns)) return true;
+    if (spin ? tc::mbar_wait_spin(bar, parity, c.wait_ns) : tc::mbar_wait(bar, parity, c.wait_ns)) return true;
     report(err, MLA_ERR_TIMEOUT);
     *c.abort_flag = 1;
     return false;
@@ -156,10 +162,11 @@ __device__ __forceinline__ int page_row(const TcParams &p, int b, int pi, int t_
 //   tm_k    3-D (64, rows, 9),    box (64, 64, 3): 64 rows x three blocks
 //   tm_v    4-D (64, rows, 4, 2), strides (1152, 128, 512), box (64, 64, 2, 2): for chunk c in
 //           {0, 1} the two blocks starting at 4c + 2 rank, i.e. columns [256c + 128 rank, +128)
-// K producer: per work item the CTA's 64 query heads (Q), then per 128-token step the CTA's own
-// page of the step.  Steps are numbered across items (g), so every slot's phase is g's parity.
+// K producers: per work item the CTA's 64 query heads (Q, the first producer only), then per
+// 128-token step K slots [j0, j1) of the CTA's own page of the step.  Steps are numbered across
+// items (g), so every slot's phase is g's parity.
 __device__ void run_k_producer(const Ctx &c, const TcParams &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
-                               int pair, int n_pairs) {
+                               int pair, int n_pairs, int j0, int j1) {
     int g = 0, item_n = 0;
     for (int k = pair; k < p.plan.n_work; k += n_pairs) {
         const WorkItem it = p.plan.items[k];
@@ -167,13 +174,15 @@ __device__ void run_k_producer(const Ctx &c, const TcParams &p, const CUtensorMa
         const int b = it.row / p.s_q;
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
         auto own_row = [&](int i) { return page_row(p, b, (it.t0 + STEP * i) / PAGE + (int)c.rank, it.t1); };
-        if (item_n > 0 && !wait_or_abort(c, c.bar(B_QEMPTY), (uint32_t)(item_n - 1) & 1u, p.err)) return;
+        if (j0 == 0) {
+            if (item_n > 0 && !wait_or_abort(c, c.bar(B_QEMPTY), (uint32_t)(item_n - 1) & 1u, p.err)) return;
+            if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_QFULL), 2u * Q_BYTES);
+            tc::tma_load_3d_pair(c.base + OFF_Q, tm_q, 0, it.row * H + 64 * (int)c.rank, 0, c.lead_bar(B_QFULL));
+        }
         ++item_n;
-        if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_QFULL), 2u * Q_BYTES);
-        tc::tma_load_3d_pair(c.base + OFF_Q, tm_q, 0, it.row * H + 64 * (int)c.rank, 0, c.lead_bar(B_QFULL));
         for (int i = 0; i < n_steps; ++i, ++g) {
             const int y = own_row(i);
-            for (int j = 0; j < NK; ++j) {
+            for (int j = j0; j < j1; ++j) {
                 if (!wait_or_abort(c, c.bar(B_KEMPTY + j), ((uint32_t)g & 1u) ^ 1u, p.err)) return;
                 if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_KFULL + j), 2u * KSLOT);
                 tc::tma_load_3d_pair(c.kslot(j), tm_k, 0, y, 3 * j, c.lead_bar(B_KFULL + j));
@@ -263,16 +272,16 @@ __device__ void run_qk_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) continue;   // only in a rejected plan, and then for every item
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
-        if (!wait_or_abort(c, c.bar(B_QFULL), (uint32_t)item_n & 1u, p.err)) return;
+        if (!wait_or_abort<true>(c, c.bar(B_QFULL), (uint32_t)item_n & 1u, p.err)) return;
         tc::fence_after_sync();
         for (int i = 0; i < n_steps; ++i, ++g) {
             const int sb = g & 1;
-            if (g >= 2 && !wait_or_abort(c, c.bar(B_SFREE + sb), (uint32_t)((g - 2) >> 1) & 1u, p.err)) return;
+            if (g >= 2 && !wait_or_abort<true>(c, c.bar(B_SFREE + sb), (uint32_t)((g - 2) >> 1) & 1u, p.err)) return;
             tc::fence_after_sync();
             const uint32_t d = tmem + TM_S + 64 * sb;
 #pragma unroll
             for (int j = 0; j < NK; ++j) {
-                if (!wait_or_abort(c, c.bar(B_KFULL + j), (uint32_t)g & 1u, p.err)) return;
+                if (!wait_or_abort<true>(c, c.bar(B_KFULL + j), (uint32_t)g & 1u, p.err)) return;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int q3 = 0; q3 < 3; ++q3)
@@ -304,16 +313,16 @@ __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
         if (it.t1 <= it.t0) continue;
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
         for (int i = 0; i < n_steps; ++i, ++g) {
-            if (!wait_or_abort(c, c.bar(B_PFULL + (g & 1)), (uint32_t)(g >> 1) & 1u, p.err)) return;
+            if (!wait_or_abort<true>(c, c.bar(B_PFULL + (g & 1)), (uint32_t)(g >> 1) & 1u, p.err)) return;
             // The first PV of an item overwrites O: the previous item's epilogue must be done with it.
-            if (i == 0 && item_n > 0 && !wait_or_abort(c, c.bar(B_OFREE), (uint32_t)(item_n - 1) & 1u, p.err)) return;
+            if (i == 0 && item_n > 0 && !wait_or_abort<true>(c, c.bar(B_OFREE), (uint32_t)(item_n - 1) & 1u, p.err)) return;
             tc::fence_after_sync();
             const uint32_t p_tmem = tmem + TM_P + 64 * (g & 1);
 #pragma unroll
             for (int pg = 0; pg < NV; ++pg) {
-                if (!wait_or_abort(c, c.bar(B_VFULL + pg), (uint32_t)g & 1u, p.err)) return;
+                if (!wait_or_abort<true>(c, c.bar(B_VFULL + pg), (uint32_t)g & 1u, p.err)) return;
                 if (ragged_rows(it, it.t0 + STEP * i + PAGE * pg) &&
-                    !wait_or_abort(c, c.bar(B_VTAIL), (uint32_t)(nt++) & 1u, p.err))
+                    !wait_or_abort<true>(c, c.bar(B_VTAIL), (uint32_t)(nt++) & 1u, p.err))
                     return;
                 tc::fence_after_sync();
 #pragma unroll
@@ -558,7 +567,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     const int pair = blockIdx.x / 2, n_pairs = gridDim.x / 2;
     if (warp == W_KPROD) {
-        if (lane == 0) run_k_producer(c, p, &tm_q, &tm_k, pair, n_pairs);
+        if (lane == 0) run_k_producer(c, p, &tm_q, &tm_k, pair, n_pairs, 0, K_SPLIT);
+    } else if (warp == W_KPROD2) {
+        if (lane == 0) run_k_producer(c, p, &tm_q, &tm_k, pair, n_pairs, K_SPLIT, NK);
     } else if (warp == W_VPROD) {
         if (lane == 0)
             run_v_producer(c, p, &tm_v, pair, n_pairs);

@@ -1,6 +1,6 @@
 """Model check of the tcgen05 absorbed decode's mbarrier protocol (decode_tc.cu), on CPU.
 
-Each role of the kernel (the K/Q producer, the V producer, the QK^T and PV issuers and the 16
+Each role of the kernel (the two K producers, the first of which also loads Q, the V producer, the QK^T and PV issuers and the 16
 softmax warps of a CTA pair) is a coroutine that yields the barrier waits it performs, in the
 kernel's order, with the kernel's slot and parity arithmetic.  mbarriers follow the hardware's
 phase rule: a wait on parity P returns once the phase of that parity has completed, so a fresh
@@ -13,6 +13,7 @@ import random
 import pytest
 
 NK, NV = 3, 2              # K ring: three slots (one step); V ring: one slot per page of a step
+K_SPLIT = 2                # K slots [0, K_SPLIT) come from the first producer, the rest from the second
 SOFTMAX_ARRIVALS = 16      # 8 softmax warps x 2 CTAs arrive on the counted barriers
 
 
@@ -63,15 +64,16 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
     k_slots, v_slots, s_buf, p_buf = [None] * NK, [None] * NV, [None, None], [None, None]
     state = {"Q": None, "O": None, "pv_done": -1}
 
-    def k_producer():
+    def k_producer(j0, j1):
         g = 0
         for n, steps in enumerate(items):
-            if n > 0:
-                yield "QEMPTY", (n - 1) & 1
-            state["Q"] = n
-            bar("QFULL").arrive()
+            if j0 == 0:
+                if n > 0:
+                    yield "QEMPTY", (n - 1) & 1
+                state["Q"] = n
+                bar("QFULL").arrive()
             for _ in range(steps):
-                for j in range(NK):
+                for j in range(j0, j1):
                     parity = (g & 1) ^ (0 if k_parity_flip else 1)
                     yield ("KEMPTY", j), parity
                     k_slots[j] = (g, j)
@@ -161,7 +163,7 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
             assert state["O"] == n, ("O", state["O"], n)
             bar("OFREE").arrive()
 
-    roles = [k_producer(), v_producer(), qk_issuer(), pv_issuer()] + \
+    roles = [k_producer(0, K_SPLIT), k_producer(K_SPLIT, NK), v_producer(), qk_issuer(), pv_issuer()] + \
         [softmax_warp() for _ in range(SOFTMAX_ARRIVALS)]
     pending = {}
     for r, co in enumerate(roles):
