@@ -117,6 +117,14 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, ui
     }
 }
 
+// One 32-byte global store (sm_100's 256-bit form): a thread writes a whole 32-byte sector, so a
+// warp storing 32 consecutive sectors writes 1 KiB of complete sectors in one instruction.
+__device__ __forceinline__ void st_global_v8(float *p, const float *v) {
+    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+                 "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
+                 : "memory");
+}
+
 // ------------------------------------------------------------------------ TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
