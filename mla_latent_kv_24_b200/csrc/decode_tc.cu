@@ -20,8 +20,8 @@
 // Every CTA loads only its own tiles, from its own GPU's HBM, with plain (non-multicast) TMA.
 //
 // Warp roles (416 threads per CTA): warps 0-7 softmax + epilogue (two warps per TMEM lane
-// quadrant, each taking half of a lane's columns), warp 8 producer of Q and of K slots 0-1,
-// warp 12 producer of K slot 2, warp 10 producer of the V ring, warp 9 QK^T issuer (leader CTA
+// quadrant, each taking half of a lane's columns), warp 8 producer of K slots 0-1, warp 12
+// producer of Q and of K slot 2, warp 10 producer of the V ring, warp 9 QK^T issuer (leader CTA
 // only) and TMEM allocator, warp 11 PV issuer (leader CTA only).  The tensor copies one thread
 // issues are processed one after another (measured: ~250 ns per copy from L2 and ~600 ns per
 // 24 KiB box from HBM under full load, whatever the ring depth), so the K ring, which streams
@@ -162,8 +162,9 @@ __device__ __forceinline__ int page_row(const TcParams &p, int b, int pi, int t_
 //   tm_k    3-D (64, rows, 9),    box (64, 64, 3): 64 rows x three blocks
 //   tm_v    4-D (64, rows, 4, 2), strides (1152, 128, 512), box (64, 64, 2, 2): for chunk c in
 //           {0, 1} the two blocks starting at 4c + 2 rank, i.e. columns [256c + 128 rank, +128)
-// K producers: per work item the CTA's 64 query heads (Q, the first producer only), then per
-// 128-token step K slots [j0, j1) of the CTA's own page of the step.  Steps are numbered across
+// K producers: per work item the CTA's 64 query heads (Q, the producer of the last slot, so Q
+// and slot 0 of an item's first step load in parallel), then per 128-token step K slots [j0, j1)
+// of the CTA's own page of the step.  Steps are numbered across
 // items (g), so every slot's phase is g's parity.
 __device__ void run_k_producer(const Ctx &c, const TcParams &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                int pair, int n_pairs, int j0, int j1) {
@@ -174,7 +175,7 @@ __device__ void run_k_producer(const Ctx &c, const TcParams &p, const CUtensorMa
         const int b = it.row / p.s_q;
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
         auto own_row = [&](int i) { return page_row(p, b, (it.t0 + STEP * i) / PAGE + (int)c.rank, it.t1); };
-        if (j0 == 0) {
+        if (j1 == NK) {
             if (item_n > 0 && !wait_or_abort(c, c.bar(B_QEMPTY), (uint32_t)(item_n - 1) & 1u, p.err)) return;
             if (c.rank == 0) tc::mbar_arrive_expect_tx(c.bar(B_QFULL), 2u * Q_BYTES);
             tc::tma_load_3d_pair(c.base + OFF_Q, tm_q, 0, it.row * H + 64 * (int)c.rank, 0, c.lead_bar(B_QFULL));

@@ -1,6 +1,6 @@
 """Model check of the tcgen05 absorbed decode's mbarrier protocol (decode_tc.cu), on CPU.
 
-Each role of the kernel (the two K producers, the first of which also loads Q, the V producer, the QK^T and PV issuers and the 16
+Each role of the kernel (the two K producers, the second of which also loads Q, the V producer, the QK^T and PV issuers and the 16
 softmax warps of a CTA pair) is a coroutine that yields the barrier waits it performs, in the
 kernel's order, with the kernel's slot and parity arithmetic.  mbarriers follow the hardware's
 phase rule: a wait on parity P returns once the phase of that parity has completed, so a fresh
@@ -67,7 +67,7 @@ def simulate(items, seed, k_parity_flip=False, skip_qempty=False, skip_pv_wait=F
     def k_producer(j0, j1):
         g = 0
         for n, steps in enumerate(items):
-            if j0 == 0:
+            if j1 == NK:
                 if n > 0:
                     yield "QEMPTY", (n - 1) & 1
                 state["Q"] = n
