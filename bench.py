@@ -39,7 +39,7 @@ UNIT = "cache tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 MAIN_KERNEL_SOURCES = {"absorbed": ["decode_tc.cu", "decode_simt.cu", "tc_ptx.cuh", "common.cuh"],
-                       "grouped": ["decode_grouped.cu", "decode_simt.cu", "warp_mma.cuh", "common.cuh"]}
+                       "grouped": ["decode_grouped.cu", "decode_simt.cu", "warp_mma.cuh", "tc_ptx.cuh", "common.cuh"]}
 
 
 def parse():

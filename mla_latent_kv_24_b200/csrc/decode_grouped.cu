@@ -7,8 +7,12 @@
 //
 // The queries arrive rotated (the q RoPE kernel runs once per call).  The path is bound by HBM
 // (8320 bytes per token for 16 groups, ~10 flop per byte per query), so the kernel streams the
-// expanded cache through a two-stage cp.async pipeline, two CTAs per SM, and uses warp-level
-// mma.sync (m16n8k16, fp32 accumulators), whose throughput is far above what the bytes need.
+// expanded cache through a two-stage pipeline of tensor copies (TMA: one 32 KiB box of K_g|V_g
+// and one 8 KiB box of k^R per page, 128-byte swizzled, completion on an mbarrier), two CTAs
+// per SM, and uses warp-level mma.sync (m16n8k16, fp32 accumulators), whose throughput is far
+// above what the bytes need.  Two tensor copies per page instead of 2,560 16-byte copies leave
+// the issue slots to the MMAs and the softmax, which matters when the SM clock drops under the
+// power limit.
 // One CTA takes one chunk of one request and one group: the group's 8 heads of every query of
 // the request form the 16 rows of the MMA tile (both MTP queries share each K/V tile), so each
 // page of K_g|V_g (32 KiB, contiguous) and of k^R (8 KiB) is read once per chunk.  Four warps
@@ -24,7 +28,11 @@
 // lives here, beside the grouped decode whose cache it reads.
 #include <math.h>
 
+#include <cudaTypedefs.h>
+#include <mutex>
+
 #include "tc_decode.h"
+#include "tc_ptx.cuh"
 #include "warp_mma.cuh"
 
 namespace mla {
@@ -32,18 +40,41 @@ namespace {
 
 constexpr int GH = 8;                 // heads per group
 constexpr int D_N = 128, D_V = 128, D_R = 64, D_QK = 192, D_LAT = 512, D_ROW = 576, PAGE = 64;
-constexpr int KV_LD = 256 + 8;        // padded [K | V] row (elements)
-constexpr int KR_LD = 64 + 8;         // padded k^R row
 constexpr int Q_LD = D_QK + 8;        // padded query row
 constexpr int STAGES = 2;
 constexpr int WARPS = 4;
-constexpr int KV_TILE = PAGE * KV_LD, KR_TILE = PAGE * KR_LD;
+// A stage holds one page: [4 blocks of 64 columns][64 rows][128 B] of K_g|V_g, then the k^R block,
+// each block 128-byte swizzled as the tensor copy writes it (16-byte chunk c of row r sits at
+// chunk c ^ (r % 8)), so the ldmatrix rows below are free of bank conflicts without padding.
+constexpr uint32_t BLK = PAGE * 128;                  // one 64-column block of a page: 8 KiB
+constexpr uint32_t KV_BYTES = 4 * BLK, KR_BYTES = BLK;
+constexpr uint32_t STAGE = KV_BYTES + KR_BYTES;       // 40 KiB
+constexpr uint32_t STAGE_BYTES = STAGES * STAGE;
 // The final cross-warp reduction reuses the stage buffers (all copies have landed by then).
-constexpr size_t STAGE_BYTES = sizeof(__nv_bfloat16) * STAGES * (KV_TILE + KR_TILE);
 constexpr size_t red_bytes(int rt) { return sizeof(float) * WARPS * 16 * rt * (2 + D_V); }
 static_assert(red_bytes(2) <= STAGE_BYTES, "reduction buffer must fit in the stage buffers");
-// 92416 B with one row tile, 98816 B with two: two CTAs per SM either way.
-constexpr size_t smem_bytes(int rt) { return STAGE_BYTES + sizeof(__nv_bfloat16) * 16 * rt * Q_LD; }
+constexpr size_t q_bytes(int rt) { return sizeof(__nv_bfloat16) * 16 * rt * Q_LD; }
+constexpr size_t bar_off(int rt) { return STAGE_BYTES + ((q_bytes(rt) + 15) & ~(size_t)15); }
+// + barriers (full and empty per stage) + room to align the window to 1024 bytes: 89 KiB with one
+// row tile, 95 KiB with two, so two CTAs per SM either way.
+constexpr size_t smem_bytes(int rt) { return 1024 + bar_off(rt) + 2 * STAGES * 8; }
+constexpr uint64_t WAIT_NS = 2000000000ull;   // 2 s: no legitimate wait comes near this
+
+// Byte offset of 16-byte chunk (row r, column c, c % 8 == 0) in a 128-byte-swizzled tile of
+// 64-column blocks of PAGE rows.
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+    return (uint32_t)((c >> 6) * BLK + r * 128 + ((((c >> 3) & 7) ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ void tma_load_3d_own(uint32_t dst, const CUtensorMap *m, int x, int y, int z, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_own(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 
 struct GParams {
     const __nv_bfloat16 *q, *expanded, *latent;   // q: rotated queries [rows, H, 192]
@@ -57,14 +88,21 @@ struct GParams {
 
 // Rows of the MMA tiles: CTA = (group g, item), row m = query m / 8 of head g*8 + m % 8; RT row
 // tiles of 16 (RT = 1 for s_q <= 2, 2 for s_q = 3, 4).
+//
+// Tensor maps (bf16, 128-byte swizzle, 64-column inner blocks):
+//   tm_kv  3-D over the expanded cache [n_pages G 64, 256]: (64, rows, 4), box (64, 64, 4): a page of K_g|V_g
+//   tm_kr  3-D over the latent cache [n_pages 64, 576]: (64, rows, 9), box (64, 64, 1) at block 8: k^R
 template <int RT>
-__global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p) {
+__global__ void __launch_bounds__(WARPS * 32, 2)
+    grouped_decode_kernel(const __grid_constant__ CUtensorMap tm_kv, const __grid_constant__ CUtensorMap tm_kr, GParams p) {
     constexpr int ROWS = 16 * RT;
     step_begin();
-    extern __shared__ __align__(16) uint8_t gsm[];
-    __nv_bfloat16 *kv = reinterpret_cast<__nv_bfloat16 *>(gsm);           // [STAGES][64][KV_LD]
-    __nv_bfloat16 *kr = kv + STAGES * KV_TILE;                            // [STAGES][64][KR_LD]
-    __nv_bfloat16 *qs = kr + STAGES * KR_TILE;                            // [ROWS][Q_LD]
+    extern __shared__ __align__(16) uint8_t gsm_raw[];
+    const uint32_t raw = smem_u32(gsm_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;                        // stages need 1024-byte alignment
+    uint8_t *gsm = gsm_raw + (sbase - raw);
+    __nv_bfloat16 *qs = reinterpret_cast<__nv_bfloat16 *>(gsm + STAGE_BYTES);   // [ROWS][Q_LD]
+    const uint32_t bars = sbase + (uint32_t)bar_off(RT);                  // full[STAGES], empty[STAGES]
     float *red_ml = reinterpret_cast<float *>(gsm);                       // [WARPS][ROWS][2], after the loop
     float *red_o = red_ml + WARPS * ROWS * 2;                             // [WARPS][ROWS][128], after the loop
 
@@ -84,6 +122,10 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
     const int n_pg = ceil_div(it.t1 - it.t0, PAGE);
     const size_t part_base = (size_t)item * p.s_q;
 
+    if (tid == 0) {
+        for (int i = 0; i < 2 * STAGES; ++i) tc::mbar_init(bars + 8 * i, i < STAGES ? 1 : WARPS);
+        tc::fence_mbar_init();
+    }
     if (it.t1 <= it.t0) {   // only in a rejected plan
         for (int m = tid; m < ROWS; m += blockDim.x) {
             if (row_query(m) >= p.s_q) continue;
@@ -104,29 +146,20 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
     }
     __syncthreads();
 
-    // Page i of the chunk into stage `stage`.  Rows past the chunk's end (the ragged last page)
-    // and the rows of an out-of-range page id are zero-filled, so stale slot contents (even
-    // non-finite ones) never reach P.V, where a zero probability would not cancel them.
-    auto load_page = [&](int stage, int i) {
+    // Page i of the chunk into stage i % STAGES (thread 0).  An out-of-range page id reads as zeros
+    // (a row coordinate past the end).  Rows past the chunk's end on its ragged last page hold
+    // whatever the slots hold, NaN included; each warp zeroes its own rows of them before use.
+    auto issue_page = [&](int i) {
         int pid = p.page_table[(size_t)b * p.max_pages + it.t0 / PAGE + i];
-        bool ok = true;
         if (pid < 0 || pid >= p.n_pages) {
-            if (tid == 0) report(p.err, MLA_ERR_DEVICE_BOUNDS);
-            ok = false;
-            pid = 0;
+            report(p.err, MLA_ERR_DEVICE_BOUNDS);
+            pid = p.n_pages;
         }
-        const int valid = ok ? min(PAGE, it.t1 - (it.t0 + PAGE * i)) : 0;
-        const __nv_bfloat16 *src_kv = p.expanded + (((size_t)pid * G + g) * PAGE) * 256;
-        const __nv_bfloat16 *src_kr = p.latent + ((size_t)pid * PAGE) * D_ROW + D_LAT;
-        __nv_bfloat16 *dkv = kv + stage * KV_TILE, *dkr = kr + stage * KR_TILE;
-        for (int c = tid; c < PAGE * 32; c += blockDim.x) {       // 64 rows x 32 chunks of 16 B
-            const int r = c / 32, k = (c % 32) * 8;
-            cp_async16(dkv + r * KV_LD + k, src_kv + (size_t)r * 256 + k, r < valid);
-        }
-        for (int c = tid; c < PAGE * 8; c += blockDim.x) {        // 64 rows x 8 chunks
-            const int r = c / 8, k = (c % 8) * 8;
-            cp_async16(dkr + r * KR_LD + k, src_kr + (size_t)r * D_ROW + k, r < valid);
-        }
+        const int st = i % STAGES;
+        const uint32_t full = bars + 8 * st, dst = sbase + STAGE * st;
+        tc::mbar_arrive_expect_tx(full, STAGE);
+        tma_load_3d_own(dst, &tm_kv, 0, (pid * G + g) * PAGE, 0, full);
+        tma_load_3d_own(dst + KV_BYTES, &tm_kr, 0, pid * PAGE, 8, full);
     };
 
     // One tile's query A fragments stay in registers for the whole chunk (12 k-steps of 16 dims);
@@ -160,15 +193,25 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
         for (int n = 0; n < 16; ++n) o[t][n][0] = o[t][n][1] = o[t][n][2] = o[t][n][3] = 0.f;
     }
 
-    load_page(0, 0);
-    cp_async_commit();
+    if (tid == 0)
+        for (int i = 0; i < STAGES && i < n_pg; ++i) issue_page(i);
+    bool ok = true;
     for (int i = 0; i < n_pg; ++i) {
-        if (i + 1 < n_pg) load_page((i + 1) % STAGES, i + 1);
-        cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
-        const __nv_bfloat16 *tkv = kv + (i % STAGES) * KV_TILE + (16 * warp) * KV_LD;
-        const __nv_bfloat16 *tkr = kr + (i % STAGES) * KR_TILE + (16 * warp) * KR_LD;
+        const int st = i % STAGES;
+        const uint32_t full = bars + 8 * st, empty = bars + 8 * (STAGES + st);
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(full, (uint32_t)(i / STAGES) & 1u, WAIT_NS));
+        if (!ok) break;
+        const uint8_t *tkv = gsm + STAGE * st, *tkr = tkv + KV_BYTES;
+        const int valid = it.t1 - (it.t0 + PAGE * i);
+        if (valid < 16 * warp + 16) {   // this warp's rows past the chunk's end: zero them
+            for (int e = lane; e < 16 * 5 * 8; e += 32) {
+                const int r = 16 * warp + e / 40, q = e % 40;   // 40 chunks of 16 B per row (4 KV blocks + k^R)
+                if (r < valid) continue;
+                uint8_t *d = const_cast<uint8_t *>(q < 32 ? tkv + (q / 8) * BLK : tkr) + r * 128 + 16 * (q % 8);
+                *reinterpret_cast<uint4 *>(d) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncwarp();
+        }
         // S [16 rows x 16 tokens] per tile = Q~ K~^T over 192 dims.
         float s[RT][2][4];
 #pragma unroll
@@ -189,9 +232,9 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 uint32_t bf[4];
-                const int tok = 8 * nt + (lane % 8);
-                const __nv_bfloat16 *src = ks < 8 ? tkv + tok * KV_LD + 16 * ks + 8 * (lane / 8)
-                                                  : tkr + tok * KR_LD + 16 * (ks - 8) + 8 * (lane / 8);
+                const int tok = 16 * warp + 8 * nt + (lane % 8);
+                const uint8_t *src = ks < 8 ? tkv + sw_off(tok, 16 * ks + 8 * (lane / 8))
+                                            : tkr + sw_off(tok, 16 * (ks - 8) + 8 * (lane / 8));
                 ldmatrix_x4(bf[0], bf[1], bf[2], bf[3], src);
 #pragma unroll
                 for (int t = 0; t < RT; ++t) {
@@ -262,7 +305,7 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
 #pragma unroll
         for (int n = 0; n < 16; n += 2) {
             uint32_t vb[4];
-            const __nv_bfloat16 *src = tkv + ((lane % 8) + 8 * ((lane / 8) % 2)) * KV_LD + D_N + 8 * n + 8 * (lane / 16);
+            const uint8_t *src = tkv + sw_off(16 * warp + (lane % 8) + 8 * ((lane / 8) % 2), D_N + 8 * n + 8 * (lane / 16));
             ldmatrix_x4_trans(vb[0], vb[1], vb[2], vb[3], src);
 #pragma unroll
             for (int t = 0; t < RT; ++t) {
@@ -270,9 +313,23 @@ __global__ void __launch_bounds__(WARPS * 32, 2) grouped_decode_kernel(GParams p
                 mma_bf16(o[t][n + 1], pa[t], vb[2], vb[3]);
             }
         }
-        __syncthreads();   // this stage is refilled by the next iteration's load
+        // This warp is done with the stage; thread 0 refills it once all four are.
+        __syncwarp();
+        if (lane == 0) mbar_arrive_own(empty);
+        if (tid == 0 && i + STAGES < n_pg) {
+            if (!tc::mbar_wait(empty, (uint32_t)(i / STAGES) & 1u, WAIT_NS)) {
+                report(p.err, MLA_ERR_TIMEOUT);
+                break;
+            }
+            issue_page(i + STAGES);
+        }
     }
-    cp_async_wait<0>();
+    if (!ok) {   // a wait ran out: let copies in flight land before the memory is released
+        if (lane == 0) report(p.err, MLA_ERR_TIMEOUT);
+        const uint64_t t0 = tc::globaltimer();
+        while (tc::globaltimer() - t0 < 200000ull) {
+        }
+    }
     __syncthreads();   // the stage buffers become the reduction buffer
 
     // Merge the four warps' partial softmaxes: row sums over the 4 threads of each row first.
@@ -352,21 +409,84 @@ static GParams grouped_params(const Dims &d, const void *q, const void *expanded
     return p;
 }
 
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiled g_encode_fn() {
+    static const EncodeTiled fn = [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<EncodeTiled>(ptr);
+        return (EncodeTiled) nullptr;
+    }();
+    return fn;
+}
+
+// The two maps of a (expanded cache, latent cache) pair; a decode loop passes the same buffers
+// every step, so recent encodings are reused (an encoding costs about a microsecond on the host).
+static bool grouped_maps(const void *expanded, const void *latent, int n_pages, int G, CUtensorMap *tm_kv,
+                         CUtensorMap *tm_kr) {
+    struct Entry {
+        const void *expanded, *latent;
+        int n_pages, G, device;
+        CUtensorMap kv, kr;
+    };
+    static std::mutex mu;
+    static Entry cache[8];
+    static int used = 0, next = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (cache[i].expanded == expanded && cache[i].latent == latent && cache[i].n_pages == n_pages &&
+                cache[i].G == G && cache[i].device == dev) {
+                *tm_kv = cache[i].kv;
+                *tm_kr = cache[i].kr;
+                return true;
+            }
+    }
+    EncodeTiled fn = g_encode_fn();
+    if (!fn) return false;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const cuuint64_t dkv[3] = {64, (cuuint64_t)n_pages * G * PAGE, 4}, skv[2] = {256 * 2, 128};
+    const cuuint32_t bkv[3] = {64, PAGE, 4};
+    const cuuint64_t dkr[3] = {64, (cuuint64_t)n_pages * PAGE, 9}, skr[2] = {D_ROW * 2, 128};
+    const cuuint32_t bkr[3] = {64, PAGE, 1};
+    if (fn(tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(expanded), dkv, skv, bkv, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+        fn(tm_kr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(latent), dkr, skr, bkr, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    std::lock_guard<std::mutex> lock(mu);
+    cache[next] = Entry{expanded, latent, n_pages, G, dev, *tm_kv, *tm_kr};
+    next = (next + 1) % 8;
+    used = used < 8 ? used + 1 : 8;
+    return true;
+}
+
 cudaError_t launch_grouped_decode(const Dims &d, const void *q, const void *expanded, const void *latent,
                                   const int *seq_lens, const int *page_table, const Plan &plan, int max_pages,
                                   int n_pages, int s_q, float *part_o, float *part_ml, int *err, cudaStream_t st) {
     if (plan.n_work == 0) return cudaSuccess;
     const GParams p = grouped_params(d, q, expanded, latent, seq_lens, page_table, plan, max_pages, n_pages, s_q,
                                      part_o, part_ml, err);
+    CUtensorMap tm_kv, tm_kr;
+    if (!grouped_maps(expanded, latent, n_pages, d.H / GH, &tm_kv, &tm_kr)) return cudaErrorInvalidValue;
     dim3 grid(d.H / GH, std::min(plan.n_work, 65535), ceil_div(plan.n_work, 65535));
     if (s_q <= 2) {
         cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<1>, smem_bytes(1));
         if (e != cudaSuccess) return e;
-        MLA_STEP_LAUNCH(grouped_decode_kernel<1>, dim3(grid), dim3(WARPS * 32), smem_bytes(1), st, p);
+        MLA_STEP_LAUNCH(grouped_decode_kernel<1>, dim3(grid), dim3(WARPS * 32), smem_bytes(1), st, tm_kv, tm_kr, p);
     } else {
         cudaError_t e = raise_smem_limit((const void *)grouped_decode_kernel<2>, smem_bytes(2));
         if (e != cudaSuccess) return e;
-        MLA_STEP_LAUNCH(grouped_decode_kernel<2>, dim3(grid), dim3(WARPS * 32), smem_bytes(2), st, p);
+        MLA_STEP_LAUNCH(grouped_decode_kernel<2>, dim3(grid), dim3(WARPS * 32), smem_bytes(2), st, tm_kv, tm_kr, p);
     }
     return cudaGetLastError();
 }
