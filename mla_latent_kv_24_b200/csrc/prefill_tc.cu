@@ -18,9 +18,10 @@
 // when it rescales O.
 // Shared memory: Q (128 queries x 192, 48 KiB), a K ring (one page per slot: 16 KiB of K_g and
 // 8 KiB of k^R) and a V ring (one step per slot: 2 pages x 64 d_v columns, 16 KiB).
-// Warp roles (256 threads): warps 0-3 softmax (thread = query row) and epilogue, warp 4 K/Q
-// producer, warp 5 QK^T issuer (leader CTA) and TMEM allocator, warp 6 V producer, warp 7 PV
-// issuer (leader CTA).  Every wait is bounded; a timeout records MLA_ERR_TIMEOUT and the kernel
+// Warp roles (384 threads): warps 0-7 softmax and epilogue (two warps per TMEM lane quadrant: a
+// query row's 128 scores of a step are split between the threads of lane L in warps w and w + 4),
+// warp 8 K/Q producer, warp 9 QK^T issuer (leader CTA) and TMEM allocator, warp 10 V producer,
+// warp 11 PV issuer (leader CTA).  Every wait is bounded; a timeout records MLA_ERR_TIMEOUT and the kernel
 // still frees its tensor memory.
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -58,7 +59,8 @@ enum {
 };
 constexpr uint32_t OFF_TMEMPTR = OFF_BAR + B_COUNT * 8;
 constexpr uint32_t OFF_FLAG = OFF_TMEMPTR + 8;
-constexpr uint32_t SMEM_USED = OFF_FLAG + 8;
+constexpr uint32_t OFF_RED = (OFF_FLAG + 8 + 15) & ~15u;   // float[2 buffers][2 halves][128 rows]
+constexpr uint32_t SMEM_USED = OFF_RED + 2 * 2 * 128 * 4;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
@@ -70,9 +72,9 @@ constexpr uint32_t TM_COLS = 512;
 constexpr uint32_t IDESC_QK = tc::idesc_bf16_f32(256, 128, false, false);
 constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(256, 128, false, true);
 constexpr uint64_t WAIT_NS = 2000000000ull;
-constexpr int SM_WARPS = 4;
-constexpr int W_KPROD = 4, W_QK = 5, W_VPROD = 6, W_PV = 7;
-constexpr int THREADS = 256;
+constexpr int SM_WARPS = 8;
+constexpr int W_KPROD = 8, W_QK = 9, W_VPROD = 10, W_PV = 11;
+constexpr int THREADS = 384;
 constexpr float RESCALE_LOG2 = 8.f;
 
 struct PfParams {
@@ -232,35 +234,44 @@ __device__ void run_pv_issuer(const Ctx &c, const PfParams &p, const Unit &u, ui
 }
 
 // --------------------------------------------------------------------------- softmax + epilogue
-// Thread L of warps 0-3 owns TMEM lane L, i.e. query q0 + 128 rank + L: its whole S row (128
-// tokens) is in its registers, so the row max and sum need no exchange.  O is rescaled lazily,
-// only when a row max grows by more than 2^8 (exact after the final division by l), decided per
-// warp so the TMEM loads stay warp-uniform.
+// Warps w and w + 4 read TMEM lane quadrant w % 4: thread L = 32 (w % 4) + lane of warp w owns
+// query q0 + 128 rank + L and tokens [64 (w / 4), +64) of each step.  The two threads of a row swap
+// their maxima through shared memory (one 64-thread named barrier per warp pair) and keep their
+// own sums, added at the end.  O is rescaled lazily, only when a row max grows by more than 2^8
+// (exact after the final division by l); both warps of a pair see the same rows and maxima, so
+// their warp-uniform rescale decisions agree.
 __device__ void run_softmax(const Ctx &c, const PfParams &p, const Unit &u, uint32_t tmem) {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int L = 32 * warp + lane;
+    const int quad = warp & 3, half = warp >> 2;
+    const int L = 32 * quad + lane;
     const int q = u.q0 + QT * (int)c.rank + L;
-    const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_addr = (uint32_t)(32 * quad) << 16;
     const int p_q = min(u.L - p.n_q + q, u.L - 1);   // last visible token (padding rows: the last token)
+    float *red = reinterpret_cast<float *>(c.sbase + OFF_RED);   // [2][2][128]
+    auto partner = [&](int buf, float v) {
+        red[256 * buf + 128 * half + L] = v;
+        tc::named_sync(1 + quad, 64);
+        return red[256 * buf + 128 * (half ^ 1) + L];
+    };
     float m_run = -INFINITY, l_run = 0.f;
     for (int i = 0; i < u.n_steps; ++i) {
         const int sb = i & 1;
         warp_wait(c, c.bar(B_SFULL + sb), (uint32_t)(i >> 1) & 1u, p.err);
         tc::fence_after_sync();
-        float s[128];
-        tc::tmem_ld64(tmem + TM_S + 128 * sb + lane_addr, s);
-        tc::tmem_ld64(tmem + TM_S + 128 * sb + 64 + lane_addr, s + 64);
+        float s[64];
+        tc::tmem_ld64(tmem + TM_S + 128 * sb + 64 * half + lane_addr, s);
         tc::tmem_wait_ld();
         tc::fence_before_sync();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive_cluster(c.lead_bar(B_SFREE + sb));
-        const int nvis = min(STEP, max(0, p_q - (u.t0 + STEP * i) + 1));   // visible prefix of the step
+        const int nvis = min(STEP, max(0, p_q - (u.t0 + STEP * i) + 1)) - 64 * half;   // visible prefix of my tokens
         float mx = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 128; ++j) {
+        for (int j = 0; j < 64; ++j) {
             s[j] = j < nvis ? s[j] * p.scale_log2 : -INFINITY;
             mx = fmaxf(mx, s[j]);
         }
+        mx = fmaxf(mx, partner(i & 1, mx));
         const bool any = __any_sync(0xffffffffu, i > 0 && mx > m_run + RESCALE_LOG2);
         // PV(i-1) must be complete before O is rescaled and before P is overwritten.
         // P is double-buffered: P(i) needs PV(i-2) complete; a rescale of O needs PV(i-1).
@@ -274,23 +285,20 @@ __device__ void run_softmax(const Ctx &c, const PfParams &p, const Unit &u, uint
         } else if (any) {
             const float m_new = fmaxf(m_run, mx);
             const float alpha = m_new == -INFINITY ? 1.f : tc::ex2(m_run - m_new);
-#pragma unroll 1
-            for (int h2 = 0; h2 < 2; ++h2) {
-                float v[64];
-                tc::tmem_ld64(tmem + TM_O + 64 * h2 + lane_addr, v);
-                tc::tmem_wait_ld();
+            float v[64];
+            tc::tmem_ld64(tmem + TM_O + 64 * half + lane_addr, v);
+            tc::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 64; ++j) v[j] *= alpha;
-                tc::tmem_st64(tmem + TM_O + 64 * h2 + lane_addr, v);
-            }
+            for (int j = 0; j < 64; ++j) v[j] *= alpha;
+            tc::tmem_st64(tmem + TM_O + 64 * half + lane_addr, v);
             tc::tmem_wait_st();
             l_run *= alpha;
             m_run = m_new;
         }
-        uint32_t pk[64];
+        uint32_t pk[32];
         float sum = 0.f;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
+        for (int j = 0; j < 32; ++j) {
             const float a = 2 * j < nvis ? tc::ex2(s[2 * j] - m_run) : 0.f;
             const float b2 = 2 * j + 1 < nvis ? tc::ex2(s[2 * j + 1] - m_run) : 0.f;
             sum += a + b2;
@@ -298,7 +306,9 @@ __device__ void run_softmax(const Ctx &c, const PfParams &p, const Unit &u, uint
             pk[j] = *reinterpret_cast<uint32_t *>(&h2);
         }
         l_run += sum;
-        tc::tmem_st64(tmem + TM_P + 64 * (i & 1) + lane_addr, reinterpret_cast<const float *>(pk));
+        const uint32_t pcol = tmem + TM_P + 64 * (i & 1) + 32 * half + lane_addr;
+        tc::tmem_st16(pcol, pk);
+        tc::tmem_st16(pcol + 16, pk + 16);
         tc::tmem_wait_st();
         tc::fence_before_sync();
         __syncwarp();
@@ -309,27 +319,25 @@ __device__ void run_softmax(const Ctx &c, const PfParams &p, const Unit &u, uint
         warp_wait(c, c.bar(B_PVDONE + ((u.n_steps - 1) & 1)), (uint32_t)((u.n_steps - 1) >> 1) & 1u, p.err);
         tc::fence_after_sync();
     }
+    const float l_tot = l_run + partner(u.n_steps & 1, l_run);
     const bool real = q < p.n_q;
     const size_t r = ((size_t)(blockIdx.z / p.H) * p.n_q + q) * p.H + u.head;
-#pragma unroll 1
-    for (int h2 = 0; h2 < 2; ++h2) {
-        float v[64];
-        if (u.n_steps > 0) {
-            tc::tmem_ld64(tmem + TM_O + 64 * h2 + lane_addr, v);
-            tc::tmem_wait_ld();
-        } else {
+    float v[64];
+    if (u.n_steps > 0) {
+        tc::tmem_ld64(tmem + TM_O + 64 * half + lane_addr, v);
+        tc::tmem_wait_ld();
+    } else {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) v[j] = 0.f;
-        }
-        if (real) {
-            float4 *dst = reinterpret_cast<float4 *>(p.part_o + r * D_V + 64 * h2);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        }
+        for (int j = 0; j < 64; ++j) v[j] = 0.f;
     }
     if (real) {
-        p.part_ml[r * 2] = m_run * 0.69314718055994531f;
-        p.part_ml[r * 2 + 1] = l_run;
+        float *dst = p.part_o + r * D_V + 64 * half;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) tc::st_global_v8(dst + 8 * j, v + 8 * j);
+        if (half == 0) {
+            p.part_ml[r * 2] = m_run * 0.69314718055994531f;
+            p.part_ml[r * 2 + 1] = l_tot;
+        }
     }
 }
 
