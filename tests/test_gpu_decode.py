@@ -201,6 +201,23 @@ def test_out_of_range_page_id_is_reported_not_faulted():
     assert_close(got, oracle_decode(inp), "bf16", "after bounds error")
 
 
+def test_grouped_out_of_range_page_id_is_reported_not_faulted():
+    # the grouped path's tensor copies read an out-of-range page as zeros and report the id
+    w = wl.small_workload(wl.WORKLOADS["5_8192_2"], B=2, lens=[200, 300], shuffle_pages=True, seed=13)
+    inp = wl.make_inputs(w)
+    dev = Dev(inp)
+    exp = dev.expand()
+    dev.page_table[0, 2] = inp.n_pages + 7
+    dev.decode_grouped(exp)
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_get_device_status()
+    assert e.value.status == 5
+    dev.page_table[0, 2] = int(inp.page_table[0, 2])      # the context stays usable
+    got = wl.from_torch_f64(dev.decode_grouped(exp))
+    mla.mla_get_device_status()
+    assert_close(got, oracle_decode(inp), "bf16", "grouped after bounds error")
+
+
 def test_device_seq_lens_disagreeing_with_host_is_reported():
     w = wl.small_workload(wl.WORKLOADS["2"], B=2, lens=[100, 300], seed=4)
     inp = wl.make_inputs(w)
