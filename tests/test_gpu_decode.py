@@ -90,9 +90,13 @@ def test_grouped_multi_chunk_shapes_match_oracle(B, s_q, lens):
     assert_close(got, oracle_decode(inp), "bf16", f"grouped multi-chunk {lens}")
 
 
-def test_grouped_ignores_nonfinite_stale_slots():
-    # slots past a request's length in its last page are never read as keys or values
-    w = wl.small_workload(wl.WORKLOADS["5_8192_1"], B=3, s_q=2, lens=[70, 130, 1000], shuffle_pages=True, seed=21)
+@pytest.mark.parametrize("s_q,lens", [(2, (70, 130, 1000)), (1, (84, 127, 1111, 64)), (4, (70, 150, 1000, 1087))])
+def test_grouped_ignores_nonfinite_stale_slots(s_q, lens):
+    # slots past a request's length in its last page are never read as keys or values: the page
+    # arrives whole by tensor copy and each warp zeroes its own rows past the end (last pages with
+    # 2 to 63 valid rows put the end inside every warp's 16-row band; s_q = 4 runs two row tiles)
+    w = wl.small_workload(wl.WORKLOADS["5_8192_1"], B=len(lens), s_q=s_q, lens=list(lens), shuffle_pages=True,
+                          seed=21 + s_q)
     inp = wl.make_inputs(w)
     dev = Dev(inp)
     exp = dev.expand()
@@ -102,7 +106,8 @@ def test_grouped_ignores_nonfinite_stale_slots():
         exp[last, :, used:, :] = float("nan")
         dev.cache.view(inp.n_pages, w.page, w.d_row)[last, used:, :] = float("nan")
     got = wl.from_torch_f64(dev.decode_grouped(exp))
-    assert_close(got, oracle_decode(inp), "bf16", "grouped with NaN stale slots")
+    mla.mla_get_device_status()
+    assert_close(got, oracle_decode(inp), "bf16", f"grouped with NaN stale slots s_q={s_q}")
 
 
 @pytest.mark.parametrize("s_q,lens", [(1, (70, 130, 1000, 64)), (2, (70, 129, 1000, 5))])
