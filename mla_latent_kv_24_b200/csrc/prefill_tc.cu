@@ -424,15 +424,16 @@ using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t,
                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Looked up once; the initialisation of a function-local static is thread-safe.
 EncodeTiled pf_encode_fn() {
-    static EncodeTiled fn = nullptr;
-    if (!fn) {
+    static const EncodeTiled fn = [] {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult qr;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
             qr == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiled>(ptr);
-    }
+            return reinterpret_cast<EncodeTiled>(ptr);
+        return (EncodeTiled) nullptr;
+    }();
     return fn;
 }
 
