@@ -137,7 +137,7 @@ mla_status check_batch(const Dims &d, int batch, int s_q, int max_pages, const i
 // item covers all s_q queries of a request (they share every K/V tile), so the plan has one
 // row per request and each item stores s_q partial results (qpi = queries per item).
 struct Layout {
-    size_t q_off, items_off, row_off, po_off, pml_off, total;
+    size_t q_off, items_off, row_off, order_off, po_off, pml_off, total;
     int n_work, chunk, rows, plan_sq, qpi, DK, DV;
     bool tc;
 };
@@ -174,6 +174,8 @@ mla_status make_layout(const Dims &d, Path path, bool tc, int sms, int batch, in
     off = align256(off + (size_t)L->n_work * sizeof(WorkItem));
     L->row_off = off;
     off = align256(off + (size_t)(batch * L->plan_sq + 1) * sizeof(int));
+    L->order_off = off;   // the tcgen05 decode's take order of the items, and the plan's scratch
+    off = align256(off + (tc ? (size_t)(L->n_work + batch * L->plan_sq + 1) * sizeof(int) : 0));
     L->po_off = off;
     off = align256(off + (size_t)L->n_work * L->qpi * d.H * L->DV * sizeof(float));
     L->pml_off = off;
@@ -328,9 +330,10 @@ static mla_status run_decode(Path path, const mla_dims *dims, const void *q, con
     float *part_o = (float *)(w + L.po_off);
     float *part_ml = (float *)(w + L.pml_off);
     void *qp = w + L.q_off;
-    Plan plan{items, row_first, L.n_work, batch * L.plan_sq, L.chunk};
+    int *order = tc ? (int *)(w + L.order_off) : nullptr;
+    Plan plan{items, row_first, L.n_work, batch * L.plan_sq, L.chunk, order};
 
-    const PlanArgs pa{seq_lens, batch, L.plan_sq, max_pages, d.page, L.chunk, L.n_work, items, row_first, err};
+    const PlanArgs pa{seq_lens, batch, L.plan_sq, max_pages, d.page, L.chunk, L.n_work, items, row_first, err, order};
     if (path == ABSORBED) {
         if (q_absorb_mma_ok(d)) {
             MLA_CUDA(launch_q_absorb_mma(d, q, W_uk, seq_lens, batch, s_q, qp, pa, st),

@@ -86,6 +86,8 @@ struct PlanArgs {
     WorkItem *items;     // [n_expected]
     int *row_first;      // [batch * s_q + 1]
     int *err;
+    int *order;          // optional: [n_expected] take order of the items (see plan_block), then
+                         // [batch * s_q + 1] scratch
 };
 
 struct Plan {
@@ -94,6 +96,7 @@ struct Plan {
     int n_work;
     int rows;
     int chunk;
+    const int *order;       // nullptr, or the order in which a persistent decode takes the items
 };
 
 }  // namespace mla

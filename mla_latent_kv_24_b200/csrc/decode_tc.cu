@@ -143,6 +143,16 @@ __device__ __forceinline__ bool warp_wait(const Ctx &c, uint32_t bar, uint32_t p
     return __all_sync(0xffffffffu, ok);
 }
 
+// Work item of round `rnd` of cluster pair `pair`: the plan's positions are dealt in snake order
+// (pairs 0..U-1, then U-1..0, ...), and the plan lists full-length chunks first and the rows'
+// shorter last chunks longest first, so every pair gets a similar number of steps even when the
+// rows' lengths differ widely.  Every role of both CTAs walks the same sequence.  -1: no more.
+__device__ __forceinline__ int item_of_round(const Plan &pl, int pair, int n_pairs, int rnd) {
+    const int j = rnd * n_pairs + ((rnd & 1) ? n_pairs - 1 - pair : pair);
+    if (j >= pl.n_work) return -1;
+    return pl.order ? pl.order[j] : j;
+}
+
 // Row coordinate (in the [n_pages*64, 576] view) of page index `pi` of request `b`; pages with
 // no token before `t_end` and out-of-range page ids read as zeros (coordinate past the end).
 __device__ __forceinline__ int page_row(const TcParams &p, int b, int pi, int t_end) {
@@ -169,7 +179,7 @@ __device__ __forceinline__ int page_row(const TcParams &p, int b, int pi, int t_
 __device__ void run_k_producer(const Ctx &c, const TcParams &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                int pair, int n_pairs, int j0, int j1) {
     int g = 0, item_n = 0;
-    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
+    for (int rnd = 0, k; (k = item_of_round(p.plan, pair, n_pairs, rnd)) >= 0; ++rnd) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) continue;   // only in a rejected plan, and then for every item
         const int b = it.row / p.s_q;
@@ -205,7 +215,7 @@ __device__ __forceinline__ int ragged_rows(const WorkItem &it, int row0) {
 // cleared by run_v_tail.
 __device__ void run_v_producer(const Ctx &c, const TcParams &p, const CUtensorMap *tm_v, int pair, int n_pairs) {
     int g = 0;
-    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
+    for (int rnd = 0, k; (k = item_of_round(p.plan, pair, n_pairs, rnd)) >= 0; ++rnd) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) continue;
         const int b = it.row / p.s_q;
@@ -237,7 +247,7 @@ __device__ void run_v_producer(const Ctx &c, const TcParams &p, const CUtensorMa
 __device__ void run_v_tail(const Ctx &c, const TcParams &p, int pair, int n_pairs) {
     const int lane = threadIdx.x % 32;   // 1..31
     int nt = 0;                          // ragged pages so far (phase of B_VLOCAL)
-    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
+    for (int rnd = 0, k; (k = item_of_round(p.plan, pair, n_pairs, rnd)) >= 0; ++rnd) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) continue;
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
@@ -269,7 +279,7 @@ __device__ void run_qk_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
     int g = 0, item_n = 0;
     const uint64_t qdesc = tc::sdesc_sw128(c.base + OFF_Q, 16, 1024);
     const uint64_t kdesc = tc::sdesc_sw128(c.base + OFF_K, 16, 1024);
-    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
+    for (int rnd = 0, k; (k = item_of_round(p.plan, pair, n_pairs, rnd)) >= 0; ++rnd) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) continue;   // only in a rejected plan, and then for every item
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
@@ -309,7 +319,7 @@ __device__ void run_pv_issuer(const Ctx &c, const TcParams &p, uint32_t tmem, in
     int g = 0, item_n = 0, nt = 0;   // nt: ragged pages so far (phase of B_VTAIL)
     const uint64_t vdesc = tc::sdesc_sw128(c.base + OFF_V, BOX, 1024);
     const uint32_t o_tmem = tmem + TM_O;
-    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
+    for (int rnd = 0, k; (k = item_of_round(p.plan, pair, n_pairs, rnd)) >= 0; ++rnd) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) continue;
         const int n_steps = ceil_div(it.t1 - it.t0, STEP);
@@ -370,7 +380,7 @@ __device__ void run_softmax(const Ctx &c, const TcParams &p, uint32_t tmem, int 
         d = r[128 * (half ^ 1) + (L ^ 64)];
     };
     int g = 0;
-    for (int k = pair; k < p.plan.n_work; k += n_pairs) {
+    for (int rnd = 0, k; (k = item_of_round(p.plan, pair, n_pairs, rnd)) >= 0; ++rnd) {
         const WorkItem it = p.plan.items[k];
         if (it.t1 <= it.t0) {
             if (hsel == 0 && half == 0) {
