@@ -313,15 +313,18 @@ __global__ void __launch_bounds__(WARPS * 32, 2)
                 mma_bf16(o[t][n + 1], pa[t], vb[2], vb[3]);
             }
         }
-        // This warp is done with the stage; thread 0 refills it once all four are.
+        // This warp is done with the stage; thread 0 refills it once all four are.  If that wait
+        // runs out, warp 0 leaves the loop as a whole (the other warps' next waits then run out).
         __syncwarp();
         if (lane == 0) mbar_arrive_own(empty);
+        bool refilled = true;
         if (tid == 0 && i + STAGES < n_pg) {
-            if (!tc::mbar_wait(empty, (uint32_t)(i / STAGES) & 1u, WAIT_NS)) {
-                report(p.err, MLA_ERR_TIMEOUT);
-                break;
-            }
-            issue_page(i + STAGES);
+            refilled = tc::mbar_wait(empty, (uint32_t)(i / STAGES) & 1u, WAIT_NS);
+            if (refilled) issue_page(i + STAGES);
+        }
+        if (warp == 0 && !__all_sync(0xffffffffu, refilled)) {
+            ok = false;
+            break;
         }
     }
     if (!ok) {   // a wait ran out: let copies in flight land before the memory is released
