@@ -51,6 +51,7 @@ def _rows(lens, s_q):
 @pytest.mark.parametrize("lens,s_q,units", [
     ([131072] * 4, 1, 74), ([4096] * 8, 1, 74), ([64], 1, 74), ([1], 1, 74), ([1, 2, 3], 2, 74),
     (list(range(1024, 1024 + 128 * 200, 200)), 2, 74), ([65536] * 32, 2, 74), ([5000, 7, 130000], 1, 3),
+    ([1024 + 997 * i % 31744 for i in range(64)], 2, 74), ([300] * 200, 1, 74),
 ])
 @pytest.mark.parametrize("granule", [32, 128])
 def test_plan_rule(probe, lens, s_q, units, granule):
@@ -66,3 +67,9 @@ def test_plan_rule(probe, lens, s_q, units, granule):
         assert count <= units, "a plan that fits one wave exists but was not chosen"
         if chunk > granule:   # and no smaller chunk would still fit
             assert sum(-(-r // (chunk - granule)) for r in rows) > units
+    else:
+        # more rows than workers: three quarters of the even split of all tokens, on the granule
+        round_up = lambda c: max(granule, -(-c // granule) * granule)
+        even = round_up(-(-sum(rows) // units))
+        if even < round_up(max(rows)):
+            assert chunk == round_up(even * 3 // 4)
