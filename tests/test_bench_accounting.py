@@ -53,3 +53,25 @@ def test_mtp_visible_pairs_are_causal():
     a = b.algorithmic(w, lens, "absorbed")
     visible = (9 + 10) + (2 + 3)                     # query j of a request sees L - s_q + j + 1 tokens
     assert a["kernel_flops"] == visible * 128 * 2 * (576 + 512)
+
+
+def test_committed_traffic_records_read_the_cache_once():
+    # each committed ncu record (profiles/traffic_*.txt) of a main kernel's DRAM bytes per launch is
+    # the algorithmic bytes plus at most 2 % (the cache is read once; the partials stay in L2)
+    b = _bench()
+    for path, key in (("absorbed", "3"), ("grouped", "5_8192_1")):
+        fn = os.path.join(ROOT, "profiles", f"traffic_{path}_{key}.txt")
+        vals = dict(line.split(":", 1) for line in open(fn) if ":" in line and not line.startswith("#"))
+        traffic = float(vals["dram_bytes_per_launch"])
+        w = b.wl.WORKLOADS[key]
+        alg = b.algorithmic(w, np.asarray(w.lens, dtype=np.int64), path)["kernel_bytes"]
+        assert 1.0 <= traffic / alg <= 1.02, (path, key, traffic, alg)
+
+
+def test_a_traffic_record_is_ignored_once_the_kernel_source_changes(monkeypatch):
+    b = _bench()
+    current = b.recorded_traffic("absorbed", "3")
+    monkeypatch.setattr(b, "source_hash", lambda names: "0000000000000000")
+    assert b.recorded_traffic("absorbed", "3") is None
+    assert b.recorded_traffic("absorbed", "no_such_workload") is None
+    assert current is None or current > 0
